@@ -1,0 +1,762 @@
+// C ABI of the lq library: argument checks, resident objects, dispatch and the
+// loop driver (CUDA-graph replay of the T x L schedule).
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <cmath>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "lq_common.cuh"
+
+namespace lq {
+
+static thread_local std::string g_err;
+
+void set_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+}
+
+lq_status cuda_error(cudaError_t e, const char* what) {
+  set_error("%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+  return LQ_ERR_CUDA;
+}
+
+}  // namespace lq
+
+using namespace lq;
+
+struct lq_wq {
+  int64_t N = 0, K = 0, G = 0;
+  uint8_t* codes4 = nullptr;   // N x K/2 packed
+  float* scales = nullptr;     // N x G
+  float* scales_t = nullptr;   // G x N (tensor-core GEMM layout)
+  uint8_t* op[2] = {nullptr, nullptr};  // N x K operand copies: [kOpInt8], [kOpE4M3]
+  int device = 0;
+  int64_t bytes = 0;
+};
+
+struct lq_layer {
+  uint64_t id = 0;
+  const lq_wq* wq = nullptr;
+  int a = 0, b = 0, T = 0, a_bits = 4;
+  float* P1 = nullptr;  // device a x a
+  float* P2 = nullptr;  // device b x b
+  std::vector<float> las;
+};
+
+namespace {
+
+std::atomic<uint64_t> g_layer_ids{1};
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+inline int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+lq_status check_bits_group(int bits, int group, bool allow8) {
+  if (group != kGroup) {
+    set_error("group size %d is not supported (only 32)", group);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  if (!(bits == 4 || (allow8 && bits == 8))) {
+    set_error("bits=%d is not supported", bits);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  return LQ_OK;
+}
+
+lq_status check_kron(int64_t K, const float* P1, int a, const float* P2, int b, bool optional) {
+  if (optional && P1 == nullptr && P2 == nullptr) {
+    if (a != 0 || b != 0) {
+      set_error("a and b must be 0 when no Kronecker factors are given");
+      return LQ_ERR_ARG;
+    }
+    return LQ_OK;
+  }
+  if (P1 == nullptr || P2 == nullptr) {
+    set_error("both Kronecker factors must be given");
+    return LQ_ERR_ARG;
+  }
+  if (a <= 0 || b <= 0) {
+    set_error("factor sizes must be positive (a=%d, b=%d)", a, b);
+    return LQ_ERR_ARG;
+  }
+  if ((int64_t)a * b != K) {
+    set_error("a*b = %d*%d != K = %lld", a, b, (long long)K);
+    return LQ_ERR_SHAPE;
+  }
+  if (a % 4 || b % 4 || a > 128 || b > 128) {
+    set_error("Kronecker factor sizes must be multiples of 4 and at most 128 (a=%d, b=%d)", a, b);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  if (rotate_smem_bytes(a, b, nullptr) == 0) {
+    set_error("Kronecker factors %dx%d, %dx%d exceed shared memory", a, a, b, b);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  return LQ_OK;
+}
+
+lq_status check_mk(int64_t M, int64_t K) {
+  if (M < 0 || K <= 0) {
+    set_error("invalid shape M=%lld K=%lld", (long long)M, (long long)K);
+    return LQ_ERR_ARG;
+  }
+  if (K % kGroup) {
+    set_error("K=%lld is not a multiple of 32", (long long)K);
+    return LQ_ERR_SHAPE;
+  }
+  if (M * K >= (int64_t)1 << 40) {
+    set_error("M*K too large");
+    return LQ_ERR_SHAPE;
+  }
+  return LQ_OK;
+}
+
+// decode-sized M runs the weight-streaming GEMV while its activation fits in shared memory
+bool use_gemv(int64_t M, int64_t K) {
+  return M <= kGemvMaxM && (size_t)M * (K / kGroup) * 40 <= 200u * 1024u;
+}
+
+int64_t ws_bytes_for(int64_t M, int64_t K) {
+  return round_up(M * K, 256) + round_up(M * (K / kGroup) * 4, 256);
+}
+
+// Graph cache of the loop driver: one instantiated graph per argument set.
+struct GraphKey {
+  const void* x;
+  int32_t dtype;
+  int64_t M;
+  std::vector<uint64_t> layer_ids;
+  int32_t T, mode;
+  float* y;
+  void* ws;
+  int64_t ws_bytes;
+  int device;
+  bool operator<(const GraphKey& o) const {
+    if (x != o.x) return x < o.x;
+    if (dtype != o.dtype) return dtype < o.dtype;
+    if (M != o.M) return M < o.M;
+    if (layer_ids != o.layer_ids) return layer_ids < o.layer_ids;
+    if (T != o.T) return T < o.T;
+    if (mode != o.mode) return mode < o.mode;
+    if (y != o.y) return y < o.y;
+    if (ws != o.ws) return ws < o.ws;
+    if (ws_bytes != o.ws_bytes) return ws_bytes < o.ws_bytes;
+    return device < o.device;
+  }
+};
+
+std::mutex g_graph_mu;
+std::map<GraphKey, cudaGraphExec_t> g_graphs;
+std::map<int, cudaStream_t> g_capture_streams;
+
+void drop_graphs_of_layer(uint64_t id) {
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  for (auto it = g_graphs.begin(); it != g_graphs.end();) {
+    bool uses = false;
+    for (uint64_t l : it->first.layer_ids) uses |= (l == id);
+    if (uses) {
+      cudaGraphExecDestroy(it->second);
+      it = g_graphs.erase(it);
+    } else {
+      ++it;
+    }
+  }
+}
+
+// Kernel timing probe (see lq_probe_enable): event pairs per kernel kind.
+struct Probe {
+  std::mutex mu;
+  bool on = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending[LQ_PROBE_KINDS];
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Probe g_probe;
+
+enum ProbeKind { kProbeRotQuant = 0, kProbeQuant = 1, kProbeGemm = 2, kProbeGemv = 3 };
+
+struct ProbeScope {
+  cudaEvent_t a = nullptr, b = nullptr;
+  int kind;
+  cudaStream_t s;
+  ProbeScope(int k, cudaStream_t st) : kind(k), s(st) {
+    std::lock_guard<std::mutex> lk(g_probe.mu);
+    if (!g_probe.on) return;
+    a = g_probe.get();
+    b = g_probe.get();
+    cudaEventRecord(a, s);
+  }
+  ~ProbeScope() {
+    if (!a) return;
+    cudaEventRecord(b, s);
+    std::lock_guard<std::mutex> lk(g_probe.mu);
+    g_probe.pending[kind].emplace_back(a, b);
+  }
+};
+
+// one application of a layer: quantize into the workspace, then GEMM / GEMV
+lq_status enqueue_linear(const void* x, int32_t x_dtype, int64_t M, const lq_layer* L, int t,
+                         float* y, void* ws, cudaStream_t s) {
+  const lq_wq* wq = L->wq;
+  const int64_t K = wq->K, N = wq->N;
+  const bool gemv = use_gemv(M, K);
+  const int opf = gemv ? kOpInt8 : (L->a_bits == 4 ? kOpE4M3 : kOpInt8);
+  uint8_t* codes = (uint8_t*)ws;
+  float* scales = (float*)((char*)ws + round_up(M * K, 256));
+  cudaError_t e;
+  {
+    ProbeScope ps(kProbeRotQuant, s);
+    e = launch_quantize(x, x_dtype, M, K, L->P1, L->a, L->P2, L->b, L->las[t], L->a_bits,
+                        (int8_t*)codes, opf, nullptr, scales, s);
+  }
+  if (e != cudaSuccess) return cuda_error(e, "quantize launch");
+  if (gemv) {
+    ProbeScope ps(kProbeGemv, s);
+    e = launch_group_gemv((const int8_t*)codes, scales, wq->codes4, wq->scales, y, M, N, K, s);
+    if (e != cudaSuccess) return cuda_error(e, "gemv launch");
+  } else {
+    ProbeScope ps(kProbeGemm, s);
+    const char* why = nullptr;
+    e = launch_group_gemm(codes, scales, wq->op[opf], wq->scales_t, y, M, N, K, opf, s, &why);
+    if (e != cudaSuccess) {
+      if (why) {
+        set_error("gemm launch: %s", why);
+        return LQ_ERR_CUDA;
+      }
+      return cuda_error(e, "gemm launch");
+    }
+  }
+  return LQ_OK;
+}
+
+lq_status check_layer_call(const lq_layer* layer, int64_t M, int32_t x_dtype) {
+  if (!layer) {
+    set_error("null layer");
+    return LQ_ERR_ARG;
+  }
+  if (x_dtype != LQ_F32 && x_dtype != LQ_BF16) {
+    set_error("unsupported x dtype %d", x_dtype);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  if (M < 0) {
+    set_error("negative M");
+    return LQ_ERR_ARG;
+  }
+  const bool gemm = !use_gemv(M, layer->wq->K);
+  if (gemm && layer->wq->op[layer->a_bits == 4 ? kOpE4M3 : kOpInt8] == nullptr) {
+    set_error("layer has no tensor-core operand copy");
+    return LQ_ERR_ARG;
+  }
+  if (gemm && layer->wq->K % 128) {
+    set_error("K=%lld must be a multiple of 128 for the tensor-core path (M > %d)",
+              (long long)layer->wq->K, kGemvMaxM);
+    return LQ_ERR_SHAPE;
+  }
+  if (M > ((int64_t)1 << 31) - 256 || layer->wq->N > ((int64_t)1 << 30)) {
+    set_error("M or N too large");
+    return LQ_ERR_SHAPE;
+  }
+  return LQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lq_last_error(void) { return g_err.c_str(); }
+
+int32_t lq_version(void) { return 100; }
+
+int64_t lq_act_scale_bytes(int64_t M, int64_t K) { return M * (K / kGroup) * 4; }
+
+lq_status lq_quantize_act(const void* d_x, int32_t x_dtype, int64_t M, int64_t K,
+                          const float* d_P1, int32_t a, const float* d_P2, int32_t b,
+                          float las_t, int32_t bits, int32_t group, int8_t* d_codes8,
+                          uint8_t* d_codes4, float* d_scales, void* stream) {
+  lq_status st;
+  if ((st = check_mk(M, K)) != LQ_OK) return st;
+  if ((st = check_bits_group(bits, group, true)) != LQ_OK) return st;
+  if ((st = check_kron(K, d_P1, a, d_P2, b, true)) != LQ_OK) return st;
+  if (x_dtype != LQ_F32 && x_dtype != LQ_BF16) {
+    set_error("unsupported x dtype %d", x_dtype);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  if (!(las_t > 0.f) || !std::isfinite(las_t)) {
+    set_error("LAS clip must be a positive finite number (got %g)", (double)las_t);
+    return LQ_ERR_ARG;
+  }
+  if (M > 0 && (d_x == nullptr || d_scales == nullptr || (d_codes8 == nullptr && d_codes4 == nullptr))) {
+    set_error("null input or output pointer");
+    return LQ_ERR_ARG;
+  }
+  if (d_codes4 && bits != 4) {
+    set_error("packed 4-bit output requested for bits=%d", bits);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(d_x) || !aligned16(d_codes8) || !aligned16(d_codes4) || !aligned16(d_scales)) {
+    set_error("input and output pointers must be 16-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  cudaError_t e = launch_quantize(d_x, x_dtype, M, K, d_P1, a, d_P2, b, las_t, bits, d_codes8,
+                                  kOpInt8, d_codes4, d_scales, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_error(e, "quantize launch");
+  return LQ_OK;
+}
+
+lq_status lq_fold_weights(const float* d_W, int64_t N, int64_t K, const float* d_Q1, int32_t a,
+                          const float* d_Q2, int32_t b, float* d_W_out, void* stream) {
+  lq_status st;
+  if (N < 0 || K <= 0) {
+    set_error("invalid shape");
+    return LQ_ERR_ARG;
+  }
+  if (K % 8) {
+    set_error("K must be a multiple of 8");
+    return LQ_ERR_SHAPE;
+  }
+  if ((st = check_kron(K, d_Q1, a, d_Q2, b, false)) != LQ_OK) return st;
+  if (N > 0 && (!d_W || !d_W_out)) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_W) || !aligned16(d_W_out)) {
+    set_error("pointers must be 16-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  if (d_W == d_W_out && N > 0) {
+    set_error("input and output may not alias");
+    return LQ_ERR_ARG;
+  }
+  cudaError_t e = launch_rotate_store(d_W, N, K, d_Q1, a, d_Q2, b, d_W_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_error(e, "fold launch");
+  return LQ_OK;
+}
+
+lq_status lq_inverse_transpose(const float* h_P, int32_t n, float* h_out) {
+  if (!h_P || !h_out || n <= 0 || n > 4096) {
+    set_error("invalid arguments");
+    return LQ_ERR_ARG;
+  }
+  // Gauss-Jordan with partial pivoting on [P | I] in float64
+  std::vector<double> A((size_t)n * n), I((size_t)n * n, 0.0);
+  for (int i = 0; i < n * n; ++i) A[i] = h_P[i];
+  for (int i = 0; i < n; ++i) I[(size_t)i * n + i] = 1.0;
+  for (int col = 0; col < n; ++col) {
+    int piv = col;
+    for (int r = col + 1; r < n; ++r)
+      if (std::fabs(A[(size_t)r * n + col]) > std::fabs(A[(size_t)piv * n + col])) piv = r;
+    if (A[(size_t)piv * n + col] == 0.0) {
+      set_error("matrix is singular");
+      return LQ_ERR_ARG;
+    }
+    if (piv != col)
+      for (int c = 0; c < n; ++c) {
+        std::swap(A[(size_t)piv * n + c], A[(size_t)col * n + c]);
+        std::swap(I[(size_t)piv * n + c], I[(size_t)col * n + c]);
+      }
+    const double d = A[(size_t)col * n + col];
+    for (int c = 0; c < n; ++c) {
+      A[(size_t)col * n + c] /= d;
+      I[(size_t)col * n + c] /= d;
+    }
+    for (int r = 0; r < n; ++r) {
+      if (r == col) continue;
+      const double f = A[(size_t)r * n + col];
+      if (f == 0.0) continue;
+      for (int c = 0; c < n; ++c) {
+        A[(size_t)r * n + c] -= f * A[(size_t)col * n + c];
+        I[(size_t)r * n + c] -= f * I[(size_t)col * n + c];
+      }
+    }
+  }
+  // out = (P^-1)^T
+  for (int i = 0; i < n; ++i)
+    for (int j = 0; j < n; ++j) h_out[(size_t)i * n + j] = (float)I[(size_t)j * n + i];
+  return LQ_OK;
+}
+
+lq_status lq_quantize_weights(const float* d_W, int64_t N, int64_t K, int32_t bits, int32_t group,
+                              int8_t* d_codes8, uint8_t* d_codes4, float* d_scales,
+                              void* stream) {
+  lq_status st;
+  if ((st = check_mk(N, K)) != LQ_OK) return st;
+  if ((st = check_bits_group(bits, group, false)) != LQ_OK) return st;
+  if (N > 0 && (!d_W || !d_scales || (!d_codes8 && !d_codes4))) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_W) || !aligned16(d_codes8) || !aligned16(d_codes4) || !aligned16(d_scales)) {
+    set_error("pointers must be 16-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  cudaError_t e = launch_quantize(d_W, LQ_F32, N, K, nullptr, 0, nullptr, 0, 1.0f, 4, d_codes8,
+                                  kOpInt8, d_codes4, d_scales, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_error(e, "weight quantize launch");
+  return LQ_OK;
+}
+
+lq_status lq_pack_weights(const float* d_W_folded, int64_t N, int64_t K, int32_t bits,
+                          int32_t group, lq_wq** out, void* stream) {
+  lq_status st;
+  if (!out) {
+    set_error("null output handle");
+    return LQ_ERR_ARG;
+  }
+  *out = nullptr;
+  if (N <= 0) {
+    set_error("N must be positive");
+    return LQ_ERR_ARG;
+  }
+  if ((st = check_mk(N, K)) != LQ_OK) return st;
+  if ((st = check_bits_group(bits, group, false)) != LQ_OK) return st;
+  if (!d_W_folded) {
+    set_error("null weight pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_W_folded)) {
+    set_error("weight pointer must be 16-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  lq_wq* w = new lq_wq();
+  w->N = N;
+  w->K = K;
+  w->G = K / kGroup;
+  cudaGetDevice(&w->device);
+  cudaError_t e;
+  const size_t b4 = (size_t)N * K / 2, bs = (size_t)N * w->G * 4;
+  if ((e = cudaMalloc(&w->codes4, b4)) != cudaSuccess ||
+      (e = cudaMalloc(&w->scales, bs)) != cudaSuccess ||
+      (e = cudaMalloc(&w->scales_t, bs)) != cudaSuccess) {
+    lq_wq_free(w);
+    set_error("cudaMalloc of %zu bytes failed: %s", b4 + 2 * bs, cudaGetErrorString(e));
+    return LQ_ERR_NOMEM;
+  }
+  w->bytes = (int64_t)(b4 + 2 * bs);
+  e = launch_quantize(d_W_folded, LQ_F32, N, K, nullptr, 0, nullptr, 0, 1.0f, 4, nullptr,
+                      kOpInt8, w->codes4, w->scales, s);
+  if (e == cudaSuccess) e = launch_transpose_f32(w->scales, N, w->G, w->scales_t, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    lq_wq_free(w);
+    return cuda_error(e, "pack weights");
+  }
+  *out = w;
+  return LQ_OK;
+}
+
+lq_status lq_wq_info(const lq_wq* wq, int64_t* N, int64_t* K, const uint8_t** d_codes4,
+                     const float** d_scales, int64_t* device_bytes) {
+  if (!wq) {
+    set_error("null handle");
+    return LQ_ERR_ARG;
+  }
+  if (N) *N = wq->N;
+  if (K) *K = wq->K;
+  if (d_codes4) *d_codes4 = wq->codes4;
+  if (d_scales) *d_scales = wq->scales;
+  if (device_bytes) *device_bytes = wq->bytes;
+  return LQ_OK;
+}
+
+void lq_wq_free(lq_wq* wq) {
+  if (!wq) return;
+  cudaFree(wq->codes4);
+  cudaFree(wq->scales);
+  cudaFree(wq->scales_t);
+  cudaFree(wq->op[0]);
+  cudaFree(wq->op[1]);
+  delete wq;
+}
+
+lq_status lq_layer_create(const lq_wq* wq, const float* d_P1, int32_t a, const float* d_P2,
+                          int32_t b, const float* h_las, int32_t T, int32_t a_bits,
+                          lq_layer** out) {
+  if (!out) {
+    set_error("null output handle");
+    return LQ_ERR_ARG;
+  }
+  *out = nullptr;
+  if (!wq || !h_las || T <= 0) {
+    set_error("null weights, null LAS clips or T <= 0");
+    return LQ_ERR_ARG;
+  }
+  lq_status st;
+  if ((st = check_kron(wq->K, d_P1, a, d_P2, b, false)) != LQ_OK) return st;
+  if (a_bits != 4 && a_bits != 8) {
+    set_error("a_bits=%d is not supported", a_bits);
+    return LQ_ERR_UNSUPPORTED;
+  }
+  for (int t = 0; t < T; ++t)
+    if (!(h_las[t] > 0.f) || !std::isfinite(h_las[t])) {
+      set_error("LAS clip %d is not a positive finite number", t);
+      return LQ_ERR_ARG;
+    }
+  lq_layer* L = new lq_layer();
+  L->id = g_layer_ids.fetch_add(1);
+  L->wq = wq;
+  L->a = a;
+  L->b = b;
+  L->T = T;
+  L->a_bits = a_bits;
+  L->las.assign(h_las, h_las + T);
+  cudaError_t e;
+  if ((e = cudaMalloc(&L->P1, (size_t)a * a * 4)) != cudaSuccess ||
+      (e = cudaMalloc(&L->P2, (size_t)b * b * 4)) != cudaSuccess) {
+    lq_layer_free(L);
+    set_error("cudaMalloc failed: %s", cudaGetErrorString(e));
+    return LQ_ERR_NOMEM;
+  }
+  if ((e = cudaMemcpy(L->P1, d_P1, (size_t)a * a * 4, cudaMemcpyDeviceToDevice)) != cudaSuccess ||
+      (e = cudaMemcpy(L->P2, d_P2, (size_t)b * b * 4, cudaMemcpyDeviceToDevice)) != cudaSuccess) {
+    lq_layer_free(L);
+    return cuda_error(e, "copy Kronecker factors");
+  }
+  // tensor-core operand copy of the weight codes (int8 for W4A8, E4M3 for W4A4)
+  const int opf = a_bits == 4 ? kOpE4M3 : kOpInt8;
+  lq_wq* w = const_cast<lq_wq*>(wq);
+  if (w->op[opf] == nullptr) {
+    uint8_t* buf = nullptr;
+    if ((e = cudaMalloc(&buf, (size_t)w->N * w->K)) != cudaSuccess) {
+      lq_layer_free(L);
+      set_error("cudaMalloc of the operand copy failed: %s", cudaGetErrorString(e));
+      return LQ_ERR_NOMEM;
+    }
+    e = launch_codes4_to_operand(w->codes4, w->N * w->K / 2, opf, buf, 0);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+    if (e != cudaSuccess) {
+      cudaFree(buf);
+      lq_layer_free(L);
+      return cuda_error(e, "operand copy");
+    }
+    w->op[opf] = buf;
+    w->bytes += w->N * w->K;
+  }
+  *out = L;
+  return LQ_OK;
+}
+
+void lq_layer_free(lq_layer* layer) {
+  if (!layer) return;
+  drop_graphs_of_layer(layer->id);
+  cudaFree(layer->P1);
+  cudaFree(layer->P2);
+  delete layer;
+}
+
+int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M) {
+  if (!layers || L <= 0 || M < 0) return -1;
+  int64_t need = 0;
+  for (int i = 0; i < L; ++i) {
+    if (!layers[i]) return -1;
+    need = std::max(need, ws_bytes_for(M, layers[i]->wq->K));
+  }
+  return need;
+}
+
+lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_layer* layer,
+                         int32_t t, float* d_y, void* d_ws, int64_t ws_bytes, void* stream) {
+  lq_status st;
+  if ((st = check_layer_call(layer, M, x_dtype)) != LQ_OK) return st;
+  if (t < 0 || t >= layer->T) {
+    set_error("loop index t=%d outside [0, %d)", t, layer->T);
+    return LQ_ERR_SHAPE;
+  }
+  if (M == 0) return LQ_OK;
+  if (!d_x || !d_y || !d_ws) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_x) || !aligned16(d_y) || ((uintptr_t)d_ws & 255u)) {
+    set_error("x and y must be 16-byte aligned and the workspace 256-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  if (ws_bytes < ws_bytes_for(M, layer->wq->K)) {
+    set_error("workspace of %lld bytes is smaller than the %lld needed", (long long)ws_bytes,
+              (long long)ws_bytes_for(M, layer->wq->K));
+    return LQ_ERR_WORKSPACE;
+  }
+  return enqueue_linear(d_x, x_dtype, M, layer, t, d_y, d_ws, (cudaStream_t)stream);
+}
+
+static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
+                               const lq_layer* const* layers, int32_t L, int32_t T, int32_t mode,
+                               float* d_y, void* d_ws, cudaStream_t s) {
+  const char* xcur = (const char*)d_x;
+  float* ycur = d_y;
+  const float* prev_y = nullptr;
+  for (int t = 0; t < T; ++t) {
+    for (int l = 0; l < L; ++l) {
+      const lq_layer* ly = layers[l];
+      const void* xin;
+      int32_t dt;
+      if (mode == LQ_OPEN) {
+        xin = xcur;
+        dt = x_dtype;
+        xcur += M * ly->wq->K * (x_dtype == LQ_BF16 ? 2 : 4);
+      } else {
+        xin = prev_y ? (const void*)prev_y : d_x;
+        dt = prev_y ? LQ_F32 : x_dtype;
+      }
+      lq_status st = enqueue_linear(xin, dt, M, ly, t, ycur, d_ws, s);
+      if (st != LQ_OK) return st;
+      prev_y = ycur;
+      ycur += M * ly->wq->N;
+    }
+  }
+  return LQ_OK;
+}
+
+lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
+                        const lq_layer* const* layers, int32_t L, int32_t T, int32_t mode,
+                        float* d_y, void* d_ws, int64_t ws_bytes, void* stream) {
+  if (!layers || L <= 0 || T <= 0) {
+    set_error("need at least one layer and one loop");
+    return LQ_ERR_ARG;
+  }
+  if (mode != LQ_OPEN && mode != LQ_CHAIN) {
+    set_error("unknown mode %d", mode);
+    return LQ_ERR_ARG;
+  }
+  lq_status st;
+  for (int l = 0; l < L; ++l) {
+    if ((st = check_layer_call(layers[l], M, x_dtype)) != LQ_OK) return st;
+    if (layers[l]->T < T) {
+      set_error("layer %d has %d LAS clips but T=%d", l, layers[l]->T, T);
+      return LQ_ERR_SHAPE;
+    }
+    if (mode == LQ_CHAIN) {
+      const int64_t next_k = layers[(l + 1) % L]->wq->K;
+      if (layers[l]->wq->N != next_k) {
+        set_error("chain mode needs N_%d == K_%d", l, (l + 1) % L);
+        return LQ_ERR_SHAPE;
+      }
+    }
+  }
+  if (M == 0) return LQ_OK;
+  if (!d_x || !d_y || !d_ws) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_x) || !aligned16(d_y) || ((uintptr_t)d_ws & 255u)) {
+    set_error("x and y must be 16-byte aligned and the workspace 256-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  if (ws_bytes < lq_workspace_bytes(layers, L, M)) {
+    set_error("workspace too small");
+    return LQ_ERR_WORKSPACE;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  // within a caller's own capture, record the kernels into it directly
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return cuda_error(e, "stream query");
+  bool probing;
+  {
+    std::lock_guard<std::mutex> lk(g_probe.mu);
+    probing = g_probe.on;
+  }
+  if (cap != cudaStreamCaptureStatusNone || probing)
+    return enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, s);
+
+  GraphKey key;
+  key.x = d_x;
+  key.dtype = x_dtype;
+  key.M = M;
+  for (int l = 0; l < L; ++l) key.layer_ids.push_back(layers[l]->id);
+  key.T = T;
+  key.mode = mode;
+  key.y = d_y;
+  key.ws = d_ws;
+  key.ws_bytes = ws_bytes;
+  cudaGetDevice(&key.device);
+
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  auto it = g_graphs.find(key);
+  if (it == g_graphs.end()) {
+    cudaStream_t cs;
+    auto sit = g_capture_streams.find(key.device);
+    if (sit == g_capture_streams.end()) {
+      if ((e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking)) != cudaSuccess)
+        return cuda_error(e, "create capture stream");
+      g_capture_streams[key.device] = cs;
+    } else {
+      cs = sit->second;
+    }
+    if ((e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal)) != cudaSuccess)
+      return cuda_error(e, "begin capture");
+    st = enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, cs);
+    cudaGraph_t g = nullptr;
+    e = cudaStreamEndCapture(cs, &g);
+    if (st != LQ_OK) {
+      if (g) cudaGraphDestroy(g);
+      return st;
+    }
+    if (e != cudaSuccess) return cuda_error(e, "end capture");
+    cudaGraphExec_t ge = nullptr;
+    e = cudaGraphInstantiate(&ge, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return cuda_error(e, "instantiate graph");
+    it = g_graphs.emplace(key, ge).first;
+  }
+  e = cudaGraphLaunch(it->second, s);
+  if (e != cudaSuccess) return cuda_error(e, "graph launch");
+  return LQ_OK;
+}
+
+lq_status lq_probe_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_probe.mu);
+  g_probe.on = on != 0;
+  return LQ_OK;
+}
+
+lq_status lq_probe_read(double* h_ms, int64_t* h_count) {
+  if (!h_ms || !h_count) {
+    set_error("null output");
+    return LQ_ERR_ARG;
+  }
+  std::lock_guard<std::mutex> lk(g_probe.mu);
+  lq_status st = LQ_OK;
+  for (int k = 0; k < LQ_PROBE_KINDS; ++k) {
+    double tot = 0.0;
+    for (auto& pr : g_probe.pending[k]) {
+      cudaError_t e = cudaEventSynchronize(pr.second);
+      float ms = 0.f;
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.first, pr.second);
+      if (e != cudaSuccess && st == LQ_OK) st = cuda_error(e, "probe event");
+      tot += ms;
+      g_probe.pool.push_back(pr.first);
+      g_probe.pool.push_back(pr.second);
+    }
+    h_ms[k] = tot;
+    h_count[k] = (int64_t)g_probe.pending[k].size();
+    g_probe.pending[k].clear();
+  }
+  return st;
+}
+
+lq_status lq_check_device(void* stream) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_error(e, "pending CUDA error");
+  return read_and_clear_device_status((cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,242 @@
+// Shared device/host helpers of the lq library (sm_100a only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lq.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "lq is written for sm_100a (B200) only"
+#endif
+
+namespace lq {
+
+constexpr int kGroup = 32;
+
+// Operand byte format of the codes a consumer kernel reads.
+enum OperandFormat : int {
+  kOpInt8 = 0,  // two's-complement int8 codes (tcgen05 kind::i8, GEMV)
+  kOpE4M3 = 1,  // the same integer codes (|q| <= 7) encoded as FP8 E4M3 (kind::f8f6f4)
+};
+
+// ---------------------------------------------------------------------------
+// host-side error text (thread-local), defined in lq_api.cu
+// ---------------------------------------------------------------------------
+void set_error(const char* fmt, ...);
+lq_status cuda_error(cudaError_t e, const char* what);
+
+// ---------------------------------------------------------------------------
+// code encoders shared by the quantize kernels
+// ---------------------------------------------------------------------------
+// E4M3 bytes of the integers 0..7: 0, 1.0x2^0, 1.0x2^1, 1.5x2^1, 1.0x2^2,
+// 1.25x2^2, 1.5x2^2, 1.75x2^2 (bias 7, 3 mantissa bits), one byte each.
+constexpr unsigned long long kE4M3Int0to7 = 0x4E4C4A4844403800ull;
+
+__device__ __forceinline__ uint32_t encode_e4m3_int(int q) {
+  uint32_t mag = (uint32_t)(q < 0 ? -q : q);
+  uint32_t byte = (uint32_t)(kE4M3Int0to7 >> (8u * mag)) & 0xFFu;
+  return byte | (q < 0 ? 0x80u : 0u);
+}
+
+__device__ __forceinline__ uint32_t encode_code_byte(int q, int opf) {
+  return opf == kOpE4M3 ? encode_e4m3_int(q) : ((uint32_t)q & 0xFFu);
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers: mbarrier, TMA, tcgen05
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.release.cta.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase.  Gives up after `limit_ns` of wall time
+// or as soon as *abort becomes non-zero; returns false in both cases (and
+// raises *abort on a timeout so the other roles of the CTA stop too).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort, int* dev_status,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      atomicExch(dev_status, (int)LQ_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D[tmem] = A[smem desc] * B[smem desc]^T (accumulate when acc != 0)
+template <int kKindI8>
+__device__ __forceinline__ void umma_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t acc) {
+  if (kKindI8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
+// TMEM lane (quadrant base + i), columns [col, col + 32).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// packed two-lane float32 arithmetic (sm_100a)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+      : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&c)));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+      : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)));
+  return d;
+}
+
+// ---------------------------------------------------------------------------
+// launch entry points implemented by the kernel files (host side)
+// ---------------------------------------------------------------------------
+int num_sms();
+
+// quantize / rotate (lq_quant.cu)
+cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, const float* P1,
+                            int a, const float* P2, int b, float c, int bits, int8_t* codes8,
+                            int opf, uint8_t* codes4, float* scales, cudaStream_t s);
+cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const float* Q1, int a,
+                                const float* Q2, int b, float* out, cudaStream_t s);
+cudaError_t launch_codes4_to_operand(const uint8_t* codes4, int64_t n_bytes, int opf,
+                                     uint8_t* out, cudaStream_t s);
+cudaError_t launch_transpose_f32(const float* in, int64_t rows, int64_t cols, float* out,
+                                 cudaStream_t s);
+size_t rotate_smem_bytes(int a, int b, int* rows_per_block);
+
+// GEMM (lq_gemm.cu)
+cudaError_t launch_group_gemm(const uint8_t* A, const float* sa, const uint8_t* B,
+                              const float* sw_t, float* y, int64_t M, int64_t N, int64_t K,
+                              int opf, cudaStream_t s, const char** why);
+lq_status read_and_clear_device_status(cudaStream_t s);
+
+// GEMV (lq_gemv.cu)
+cudaError_t launch_group_gemv(const int8_t* qa, const float* sa, const uint8_t* w4,
+                              const float* sw, float* y, int64_t M, int64_t N, int64_t K,
+                              cudaStream_t s);
+constexpr int kGemvMaxM = 16;
+
+}  // namespace lq

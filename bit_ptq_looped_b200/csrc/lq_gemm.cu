@@ -1,0 +1,396 @@
+// Group-rescaled integer GEMM on the 5th-generation tensor cores (sm_100a).
+//
+//   y[m,n] = sum_g s_a[m,g] s_w[n,g] sum_{k in g} q_a[m,k] q_w[n,k],  g = 32-wide K groups
+//
+// ("paper_specification.yaml" of the LoopQ reproduction: lq1_quantization,
+// weights and activations group-wise with group size 32, W4 with A4/A8.)
+//
+// One CTA owns a 128 x 128 tile of y.  Each 32-wide K group is exactly one
+// tcgen05.mma instruction (K = 32 bytes for 8-bit operands), written to its
+// own TMEM accumulator, because the next group carries different scales and
+// cannot be summed into it.  Four 128-column accumulators rotate through the
+// 512 TMEM columns, so the tensor core runs up to three groups ahead of the
+// epilogue, which folds every group into float32 registers:
+//   y += (s_a[m,g] * s_w[n,g]) * acc_g[m,n].
+//
+// Operands:
+//   W4A4: codes stored as FP8 E4M3 bytes (|q| <= 7 is exact in E4M3) and
+//         multiplied with kind::f8f6f4, whose float32 accumulator holds the
+//         integer group sum (|acc| <= 32*49) exactly;
+//   W4A8: codes stored as int8 and multiplied with kind::i8 (int32 sums).
+//
+// Warp roles (320 threads): warps 0-7 epilogue (warp w reads TMEM lane
+// quadrant w % 4, column half w / 4), warp 8 TMA producer, warp 9 MMA issuer.
+// Every mbarrier wait is bounded; on expiry the kernel records
+// LQ_ERR_DEVICE_TIMEOUT in a device status word, stops all roles, frees its
+// TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "lq_common.cuh"
+
+namespace lq {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int BK = 128;                 // K elements (bytes) per pipeline stage
+constexpr int GPS = BK / kGroup;        // groups per stage = 4
+constexpr int STAGES = 5;
+constexpr int ACC_BUFS = 4;             // 4 x 128 TMEM columns
+constexpr int TMEM_COLS = 512;
+constexpr int EPI_WARPS = 8;
+constexpr int WARP_TMA = 8;
+constexpr int WARP_MMA = 9;
+constexpr int THREADS = 320;
+constexpr int EPI_COLS = BN / 2;        // columns per epilogue warp
+
+constexpr uint32_t A_BYTES = BM * BK;          // 16 KB
+constexpr uint32_t B_BYTES = BN * BK;          // 16 KB
+constexpr uint32_t SA_BYTES = BM * GPS * 4;    // 2 KB  [BM][4] float
+constexpr uint32_t SW_BYTES = GPS * BN * 4;    // 2 KB  [4][BN] float
+constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + SA_BYTES + SW_BYTES;
+
+constexpr uint32_t OFF_A = 0;
+constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr uint32_t OFF_SA = OFF_B + STAGES * B_BYTES;
+constexpr uint32_t OFF_SW = OFF_SA + STAGES * SA_BYTES;
+constexpr uint32_t OFF_BAR = OFF_SW + STAGES * SW_BYTES;
+constexpr uint32_t N_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
+constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;
+constexpr uint32_t SMEM_USED = OFF_MISC + 16;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+__device__ int g_gemm_status = 0;
+
+// Bounded wait that ignores the abort flag: used at teardown so that no bulk
+// copy or MMA of this CTA is still in flight when it exits.
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicExch(&g_gemm_status, (int)LQ_ERR_DEVICE_TIMEOUT);
+      return;
+    }
+  }
+}
+
+// K-major operand tile, 128-byte rows, 128-byte swizzle, 8-row atoms 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address (16-byte units)
+  d |= (uint64_t)1u << 16;                  // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024u >> 4) << 32;        // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1u << 46;                  // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;                  // layout: 128-byte swizzle
+  return d;
+}
+
+template <int kKindI8>
+__host__ __device__ constexpr uint32_t instr_desc() {
+  // bits: [4,6) D format, [7,10) A format, [10,13) B format, 15/16 A/B major
+  // (0 = K-major), [17,23) N >> 3, [24,29) M >> 4
+  return (kKindI8 ? (2u << 4) | (1u << 7) | (1u << 10)   // S32 <- s8 x s8
+                  : (1u << 4) | (0u << 7) | (0u << 10))  // F32 <- e4m3 x e4m3
+         | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+template <int kKindI8>
+__device__ __forceinline__ float acc_to_f32(uint32_t r) {
+  if (kKindI8) {
+    // exact int32 -> float32 for |acc| < 2^22: place it in the mantissa of 1.5 * 2^23
+    return __int_as_float((int)r + 0x4B400000) - 12582912.0f;
+  } else {
+    return __uint_as_float(r);
+  }
+}
+
+template <int kKindI8>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_group_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSW,
+                 float* __restrict__ y, int M, int N, int G) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.y * BM;
+  const int n_kb = G / GPS;
+
+  const uint32_t bar_full = base + OFF_BAR;
+  const uint32_t bar_empty = bar_full + STAGES * 8;
+  const uint32_t bar_accf = bar_empty + STAGES * 8;
+  const uint32_t bar_acce = bar_accf + ACC_BUFS * 8;
+  const uint32_t bar_drain = bar_acce + ACC_BUFS * 8;  // all MMAs of this CTA retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1 + EPI_WARPS);
+    }
+    for (int b = 0; b < ACC_BUFS; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, EPI_WARPS);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_TMA && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSA);
+    prefetch_tmap(&tmSW);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == WARP_TMA) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < n_kb; ++kb) {
+        const int st = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait_bounded(bar_empty + 8 * st, ph ^ 1u, abort_flag, &g_gemm_status,
+                               kWaitLimitNs))
+          break;
+        const uint32_t full = bar_full + 8 * st;
+        mbar_arrive_expect_tx(full, STAGE_TX);
+        tma_load_2d(base + OFF_A + st * A_BYTES, &tmA, full, kb * BK, m0);
+        tma_load_2d(base + OFF_B + st * B_BYTES, &tmB, full, kb * BK, n0);
+        tma_load_2d(base + OFF_SA + st * SA_BYTES, &tmSA, full, kb * GPS, m0);
+        tma_load_2d(base + OFF_SW + st * SW_BYTES, &tmSW, full, n0, kb * GPS);
+        issued = kb + 1;
+      }
+      // never leave the CTA with bulk copies in flight: wait (bounded, even
+      // after an abort) for the last STAGES loads to land
+      for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
+        mbar_wait_drain(bar_full + 8 * (kb % STAGES), (uint32_t)(kb / STAGES) & 1u);
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc<kKindI8>();
+      int gi = 0;  // running group index
+      bool ok = true;
+      for (int kb = 0; kb < n_kb && ok; ++kb) {
+        const int st = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait_bounded(bar_full + 8 * st, ph, abort_flag, &g_gemm_status, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_st = base + OFF_A + st * A_BYTES;
+        const uint32_t b_st = base + OFF_B + st * B_BYTES;
+        for (int j = 0; j < GPS; ++j, ++gi) {
+          const int buf = gi % ACC_BUFS;
+          const uint32_t aph = (uint32_t)(gi / ACC_BUFS) & 1u;
+          if (!mbar_wait_bounded(bar_acce + 8 * buf, aph ^ 1u, abort_flag, &g_gemm_status,
+                                 kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // one MMA per 32-wide group: advance 32 bytes inside the swizzled 128-byte rows
+          umma_ss<kKindI8>(tmem_base + (uint32_t)(buf * BN), sw128_kmajor_desc(a_st + 32u * j),
+                           sw128_kmajor_desc(b_st + 32u * j), idesc, 0u);
+          umma_commit(bar_accf + 8 * buf);
+        }
+        if (ok) umma_commit(bar_empty + 8 * st);
+      }
+      // retire every MMA of this CTA before TMEM is released
+      umma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0u);
+    }
+  } else {
+    // ---------------- epilogue: warps 0..7 ----------------
+    const int quad = warp & 3;
+    const int col0 = (warp >> 2) * EPI_COLS;
+    const int row = quad * 32 + lane;
+    float acc[EPI_COLS];
+#pragma unroll
+    for (int i = 0; i < EPI_COLS; ++i) acc[i] = 0.f;
+    int gi = 0;
+    bool ok = true;
+    for (int kb = 0; kb < n_kb && ok; ++kb) {
+      const int st = kb % STAGES;
+      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+      if (!mbar_wait_bounded(bar_full + 8 * st, ph, abort_flag, &g_gemm_status, kWaitLimitNs)) {
+        ok = false;
+        break;
+      }
+      const float4 sa4 =
+          *reinterpret_cast<const float4*>(gbase + OFF_SA + st * SA_BYTES + row * 16);
+      const float sa[GPS] = {sa4.x, sa4.y, sa4.z, sa4.w};
+      const float* sw_st = reinterpret_cast<const float*>(gbase + OFF_SW + st * SW_BYTES);
+#pragma unroll
+      for (int j = 0; j < GPS; ++j, ++gi) {
+        const int buf = gi % ACC_BUFS;
+        const uint32_t aph = (uint32_t)(gi / ACC_BUFS) & 1u;
+        if (!mbar_wait_bounded(bar_accf + 8 * buf, aph, abort_flag, &g_gemm_status,
+                               kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        const uint32_t taddr =
+            tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN + col0);
+        tmem_ld_32x32b_x32(taddr, r0);
+        tmem_ld_32x32b_x32(taddr + 32u, r1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
+        const float s = sa[j];
+        const float4* swv = reinterpret_cast<const float4*>(sw_st + j * BN + col0);
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 w = swv[c4];
+          acc[4 * c4 + 0] = fmaf(s * w.x, acc_to_f32<kKindI8>(r0[4 * c4 + 0]), acc[4 * c4 + 0]);
+          acc[4 * c4 + 1] = fmaf(s * w.y, acc_to_f32<kKindI8>(r0[4 * c4 + 1]), acc[4 * c4 + 1]);
+          acc[4 * c4 + 2] = fmaf(s * w.z, acc_to_f32<kKindI8>(r0[4 * c4 + 2]), acc[4 * c4 + 2]);
+          acc[4 * c4 + 3] = fmaf(s * w.w, acc_to_f32<kKindI8>(r0[4 * c4 + 3]), acc[4 * c4 + 3]);
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 w = swv[8 + c4];
+          acc[32 + 4 * c4 + 0] =
+              fmaf(s * w.x, acc_to_f32<kKindI8>(r1[4 * c4 + 0]), acc[32 + 4 * c4 + 0]);
+          acc[32 + 4 * c4 + 1] =
+              fmaf(s * w.y, acc_to_f32<kKindI8>(r1[4 * c4 + 1]), acc[32 + 4 * c4 + 1]);
+          acc[32 + 4 * c4 + 2] =
+              fmaf(s * w.z, acc_to_f32<kKindI8>(r1[4 * c4 + 2]), acc[32 + 4 * c4 + 2]);
+          acc[32 + 4 * c4 + 3] =
+              fmaf(s * w.w, acc_to_f32<kKindI8>(r1[4 * c4 + 3]), acc[32 + 4 * c4 + 3]);
+        }
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty + 8 * st);
+    }
+    const int gm = m0 + row;
+    if (ok && gm < M) {
+      float* yr = y + (size_t)gm * N + n0 + col0;
+#pragma unroll
+      for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
+        if (n0 + col0 + 4 * c4 < N)
+          *reinterpret_cast<float4*>(yr + 4 * c4) =
+              make_float4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle sw) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int kKindI8>
+cudaError_t launch_impl(const uint8_t* A, const float* sa, const uint8_t* B, const float* sw_t,
+                        float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                        const char** why) {
+  const int64_t G = K / kGroup;
+  CUtensorMap mA, mB, mSA, mSW;
+  if (!make_map_2d(&mA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, BK, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, BK, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mSA, sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, G, M, G * 4, GPS, BM,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&mSW, sw_t, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, G, N * 4, BN, GPS,
+                   CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    if (why) *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  static uint64_t attr_set_mask = 0;  // one bit per device
+  auto* k = k_group_gemm<kKindI8>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!((attr_set_mask >> (dev & 63)) & 1u)) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set_mask |= 1ull << (dev & 63);
+  }
+  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  k<<<grid, THREADS, SMEM_BYTES, s>>>(mA, mB, mSA, mSW, y, (int)M, (int)N, (int)G);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_group_gemm(const uint8_t* A, const float* sa, const uint8_t* B,
+                              const float* sw_t, float* y, int64_t M, int64_t N, int64_t K,
+                              int opf, cudaStream_t s, const char** why) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  if (opf == kOpE4M3) return launch_impl<0>(A, sa, B, sw_t, y, M, N, K, s, why);
+  return launch_impl<1>(A, sa, B, sw_t, y, M, N, K, s, why);
+}
+
+lq_status read_and_clear_device_status(cudaStream_t s) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error(e, "stream synchronize");
+  int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_gemm_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_error(e, "read device status");
+  if (v != 0) {
+    e = cudaMemcpyToSymbol(g_gemm_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_error(e, "clear device status");
+    set_error("a bounded device-side wait expired (status %d)", v);
+    return (lq_status)v;
+  }
+  return LQ_OK;
+}
+
+}  // namespace lq

@@ -211,6 +211,23 @@ def module_params(wl: Workload) -> List[ModuleParams]:
     return out
 
 
+def device_loop_input(wl: Workload, lin: Linear, t: int, device="cuda"):
+    """Large-workload variant of ``loop_input`` drawn on the device with torch's
+    generator (same recipe, different random stream).  Tests copy the rows
+    they check back to the host and feed those to the oracle."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([wl.seed, _TAG_ACT, lin.input_key,
+                                              lin.K]).generate_state(1)[0]))
+    x = torch.randn((wl.M, lin.K), generator=g, device=device, dtype=torch.float32)
+    ch = torch.from_numpy(outlier_channels(lin.K, wl.outlier_frac, wl.seed, lin.input_key))
+    x[:, ch.to(device)] *= torch.tensor(wl.outlier_mult, dtype=torch.float32, device=device)
+    x = x * torch.tensor(1.0 + 0.25 * t, dtype=torch.float32, device=device)
+    x = x + torch.tensor(float(np.float32(0.1 * t)), dtype=torch.float32, device=device)
+    return x.to(torch.bfloat16) if wl.x_dtype == "bf16" else x
+
+
 def random_uniform(shape, lo: float, hi: float, seed: int, *key: int) -> np.ndarray:
     return _rng(seed, 99, *key).uniform(lo, hi, size=shape).astype(np.float32)
 

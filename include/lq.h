@@ -1,0 +1,221 @@
+/*
+ * lq.h -- C ABI of the B200 (sm_100a) LoopQ-style quantized looped linear.
+ *
+ * One quantized shared linear is applied at every loop t of a depth-recurrent
+ * transformer.  At each call a token row x (length K) is
+ *   1. rotated by a Kronecker transform, x~ = x (P1 kron P2), P1 a x a,
+ *      P2 b x b, K = a*b ("paper_specification.yaml" of the LoopQ
+ *      reproduction: loopq_components.shared_transformed_backbone, Section 2
+ *      Eqs. (2)-(3); implementation_status.lq3, shared Kronecker transform);
+ *   2. split into groups of 32 consecutive elements along K, each with the
+ *      step s = fl32(fl32(c * absmax) / q_max), where c = c_{t,l} is the
+ *      per-module, per-loop LAS clip (loopq_components.las, Section 4.1;
+ *      implementation_status.lq2, clip scalars on dynamic token/group absmax
+ *      scales; lq1_quantization.granularity, group size 32);
+ *   3. quantized by symmetric round-to-nearest (ties to even):
+ *      q = clip(rne(fl32(x~ / s)), -q_max, q_max), q_max = 7 (4-bit) or 127
+ *      (8-bit), q = 0 where s = 0 (lq1_quantization.equation, Section 2
+ *      Eq. (4): Q_a(x; c) = c clip(round(x / c), q_min, q_max); Section 5.1
+ *      RTN; the bounds, tie rule and scale estimator are the paper's
+ *      underspecified items, read as stated here);
+ *   4. multiplied with group-32 4-bit weight codes:
+ *      y[m,n] = sum_g s_a[m,g] s_w[n,g] sum_{k in g} q_a[m,k] q_w[n,k].
+ * Weights are folded offline, W~ = W (P1^-T kron P2^-T) (inverse-transpose
+ * folding, implementation_status.lq3), and quantized with s_w = fl32(absmax/7).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* are CUDA device pointers of the current device;
+ *     h_* are host pointers.  `stream` is a cudaStream_t (NULL = legacy
+ *     default stream).  Work is enqueued on `stream` and the call returns
+ *     without synchronising, unless stated otherwise.
+ *   - Matrices are dense row-major with no padding between rows.
+ *   - Inputs are never modified.  The caller owns every buffer it passes.
+ *   - Every call returns an lq_status; no call aborts or throws.  On error
+ *     nothing has been enqueued and lq_last_error() (thread-local) holds a
+ *     one-line message.
+ *   - Inputs must be finite; results for NaN/Inf inputs are unspecified.
+ */
+#ifndef LQ_H_
+#define LQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t lq_status;
+
+#define LQ_OK                  0
+#define LQ_ERR_ARG             1  /* null pointer, non-positive size, c <= 0   */
+#define LQ_ERR_SHAPE           2  /* K % 32 != 0, K != a*b, N/K mismatch, t >= T */
+#define LQ_ERR_UNSUPPORTED     3  /* bits not in {4,8}, group != 32, dtype      */
+#define LQ_ERR_ALIGN           4  /* pointer not 16-byte aligned                */
+#define LQ_ERR_CUDA            5  /* CUDA launch or runtime error               */
+#define LQ_ERR_DEVICE_TIMEOUT  6  /* a bounded device-side wait expired         */
+#define LQ_ERR_NOMEM           7  /* device allocation failed                   */
+#define LQ_ERR_WORKSPACE       8  /* workspace too small                        */
+
+/* element types of activation inputs */
+#define LQ_F32   0
+#define LQ_BF16  1
+
+/* lq_loop_stack modes */
+#define LQ_OPEN  0  /* every (t, l) reads its own input                       */
+#define LQ_CHAIN 1  /* y of step (t, l) is the input of the next step          */
+
+typedef struct lq_wq lq_wq;        /* resident quantized weights (library-owned) */
+typedef struct lq_layer lq_layer;  /* weights + P factors + LAS clips of one module */
+
+/* Thread-local text of the last error (empty string if none). */
+const char* lq_last_error(void);
+
+/* ABI version: 100 * major + minor. */
+int32_t lq_version(void);
+
+/* Bytes of the scale array for an M x K activation: M * (K/32) * 4. */
+int64_t lq_act_scale_bytes(int64_t M, int64_t K);
+
+/*
+ * lq_quantize_act -- rotate (optional) and group-quantize an activation.
+ *
+ * Steps 1-3 above for every row of d_x.
+ *   d_x      M x K, element type x_dtype (LQ_F32 or LQ_BF16), 16-byte aligned.
+ *   d_P1     a x a float32 (row-major) and d_P2 b x b float32, with a*b == K,
+ *            a and b multiples of 4 and at most 128.  Pass d_P1 = d_P2 = NULL,
+ *            a = b = 0 to skip the rotation (d_x is then the transformed
+ *            input x~ itself).  The rotation accumulates in float64 and rounds
+ *            once to float32.
+ *   las_t    the LAS clip c_{t,l} > 0 of this module and loop.
+ *   bits     4 or 8 (q_max 7 or 127).  group must be 32.
+ *   d_codes8 out: M x K int8 codes (may be NULL if d_codes4 is given).
+ *   d_codes4 out: M x K/2 bytes of packed 4-bit codes, element 2j in bits 3..0
+ *            and element 2j+1 in bits 7..4, two's complement; bits must be 4
+ *            (may be NULL).
+ *   d_scales out: M x (K/32) float32 steps s_a, row-major.
+ * Errors: LQ_ERR_ARG, LQ_ERR_SHAPE (K % 32, a*b != K), LQ_ERR_UNSUPPORTED,
+ *         LQ_ERR_ALIGN (outputs must be 16-byte aligned), LQ_ERR_CUDA.
+ */
+lq_status lq_quantize_act(const void* d_x, int32_t x_dtype, int64_t M, int64_t K,
+                          const float* d_P1, int32_t a, const float* d_P2, int32_t b,
+                          float las_t, int32_t bits, int32_t group,
+                          int8_t* d_codes8, uint8_t* d_codes4, float* d_scales,
+                          void* stream);
+
+/*
+ * lq_fold_weights -- W_out = W (Q1 kron Q2), float64 accumulation, one
+ * rounding to float32.  For the inverse-transpose fold pass Q = P^-T (for an
+ * orthogonal P that is P itself; lq_inverse_transpose computes it).
+ *   d_W, d_W_out  N x K float32 (may not alias);  d_Q1 a x a, d_Q2 b x b float32.
+ */
+lq_status lq_fold_weights(const float* d_W, int64_t N, int64_t K,
+                          const float* d_Q1, int32_t a, const float* d_Q2, int32_t b,
+                          float* d_W_out, void* stream);
+
+/*
+ * lq_inverse_transpose -- host helper: h_out = (h_P^-1)^T for an n x n float32
+ * matrix, Gauss-Jordan elimination with partial pivoting in float64, rounded
+ * to float32.  Synchronous, host memory only.  LQ_ERR_ARG if P is singular.
+ */
+lq_status lq_inverse_transpose(const float* h_P, int32_t n, float* h_out);
+
+/*
+ * lq_quantize_weights -- group-32 4-bit RTN of folded weights into caller
+ * buffers: s_w[n,g] = fl32(absmax / 7), q_w = clip(rne(fl32(w / s_w)), -7, 7).
+ *   d_W        N x K float32 (already folded).  bits must be 4, group 32.
+ *   d_codes8   out N x K int8 (may be NULL);  d_codes4 out N x K/2 packed (may be NULL).
+ *   d_scales   out N x (K/32) float32, row-major.
+ */
+lq_status lq_quantize_weights(const float* d_W, int64_t N, int64_t K, int32_t bits,
+                              int32_t group, int8_t* d_codes8, uint8_t* d_codes4,
+                              float* d_scales, void* stream);
+
+/*
+ * lq_pack_weights -- quantize folded weights into a library-owned resident
+ * object used by every loop.  Allocates device memory (cudaMalloc); the call
+ * synchronises `stream` before returning.  Release with lq_wq_free.
+ * Resident layout: packed 4-bit codes N x K/2, scales N x G and G x N
+ * (float32), and the tensor-core operand copy created by lq_layer_create.
+ */
+lq_status lq_pack_weights(const float* d_W_folded, int64_t N, int64_t K, int32_t bits,
+                          int32_t group, lq_wq** out, void* stream);
+
+/*
+ * lq_wq_info -- shapes and device pointers of a resident weight object.
+ *   d_codes4 packed codes N x K/2;  d_scales N x (K/32) float32 row-major;
+ *   device_bytes: total device memory the object holds.  Any out pointer may be NULL.
+ */
+lq_status lq_wq_info(const lq_wq* wq, int64_t* N, int64_t* K, const uint8_t** d_codes4,
+                     const float** d_scales, int64_t* device_bytes);
+void lq_wq_free(lq_wq* wq);
+
+/*
+ * lq_layer_create -- bind resident weights to a module's Kronecker factors
+ * and LAS clips.  Copies P1 (a x a), P2 (b x b) (device pointers) and
+ * h_las[T] (host, every entry > 0) into library-owned device memory and
+ * prepares the tensor-core operand copy of the weights for a_bits (4 or 8).
+ * Synchronous.  `wq` must outlive the layer.  a*b must equal wq's K.
+ */
+lq_status lq_layer_create(const lq_wq* wq, const float* d_P1, int32_t a, const float* d_P2,
+                          int32_t b, const float* h_las, int32_t T, int32_t a_bits,
+                          lq_layer** out);
+void lq_layer_free(lq_layer* layer);
+
+/*
+ * Device workspace needed by lq_loop_linear / lq_loop_stack for M tokens
+ * through the given layers (the activation codes and steps of one step).
+ */
+int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M);
+
+/*
+ * lq_loop_linear -- one application of a shared quantized linear at loop t:
+ * y = Q(x (P1 kron P2); c_t) (*) Wq, steps 1-4 above.
+ *   d_x   M x K (x_dtype LQ_F32 or LQ_BF16);  d_y out M x N float32.
+ *   d_ws  workspace of at least lq_workspace_bytes(&layer, 1, M) bytes,
+ *         256-byte aligned; its contents are scratch.
+ * Errors: LQ_ERR_SHAPE if t is not in [0, T), LQ_ERR_WORKSPACE, ...
+ */
+lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_layer* layer,
+                         int32_t t, float* d_y, void* d_ws, int64_t ws_bytes, void* stream);
+
+/*
+ * lq_loop_stack -- the whole T x L loop schedule with resident weights:
+ * for t = 0..T-1, for l = 0..L-1: y_{t,l} = lq_loop_linear(x_{t,l}, layer l, t).
+ *   mode LQ_OPEN : d_x holds T*L inputs, ordered (t, l), each M x K_l of x_dtype.
+ *   mode LQ_CHAIN: d_x holds one M x K_0 input; x_{t,l} is the previous
+ *                  step's y (float32).  Needs N_l == K_{l+1} and N_{L-1} == K_0.
+ *   d_y   out: T*L outputs ordered (t, l), each M x N_l float32.
+ * The schedule is recorded once into a CUDA graph per distinct argument set
+ * and replayed (when `stream` is itself capturing, kernels are launched
+ * directly into the caller's capture instead).
+ */
+lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
+                        const lq_layer* const* layers, int32_t L, int32_t T, int32_t mode,
+                        float* d_y, void* d_ws, int64_t ws_bytes, void* stream);
+
+/*
+ * Kernel timing probe.  While enabled (on != 0), lq_loop_linear and
+ * lq_loop_stack launch their kernels directly (no graph) and bracket each one
+ * with CUDA events recorded on the launching stream.  lq_probe_read waits for
+ * those events and returns, per kernel kind, the summed device time in
+ * milliseconds and the number of launches, then clears them.  Kinds (index):
+ * 0 fused rotate+quantize, 1 quantize-only, 2 tensor-core GEMM, 3 GEMV.
+ * h_ms and h_count point to arrays of LQ_PROBE_KINDS entries (host memory).
+ */
+#define LQ_PROBE_KINDS 4
+lq_status lq_probe_enable(int32_t on);
+lq_status lq_probe_read(double* h_ms, int64_t* h_count);
+
+/*
+ * lq_check_device -- synchronise `stream`, then read and clear the device
+ * status word that kernels set when a bounded wait expires.  Returns LQ_OK or
+ * LQ_ERR_DEVICE_TIMEOUT (or LQ_ERR_CUDA for an asynchronous CUDA error).
+ */
+lq_status lq_check_device(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LQ_H_ */

@@ -63,8 +63,8 @@ def qmax_for_bits(bits: int) -> int:
 # Kronecker transform (shared transformed backbone, Section 2 Eqs. (2)-(3);
 # implementation_status.lq3)
 # --------------------------------------------------------------------------
-def kron_rotate(x: np.ndarray, P1: np.ndarray, P2: np.ndarray) -> np.ndarray:
-    """x~ = x (P1 kron P2) for every row of x, float64 arithmetic, rounded once to float32.
+def kron_rotate_f64(x: np.ndarray, P1: np.ndarray, P2: np.ndarray) -> np.ndarray:
+    """x (P1 kron P2) for every row of x in float64 (not rounded).
 
     With the row-major reshape X = x.reshape(a, b) (index k = i*b + j), the
     product x (P1 kron P2) equals vec(P1^T X P2).
@@ -76,7 +76,12 @@ def kron_rotate(x: np.ndarray, P1: np.ndarray, P2: np.ndarray) -> np.ndarray:
     X = x.reshape(M, a, b)
     Z = np.einsum("pi,mpq,qj->mij", np.asarray(P1, np.float64), X,
                   np.asarray(P2, np.float64), optimize=True)
-    return Z.reshape(M, K).astype(np.float32)
+    return Z.reshape(M, K)
+
+
+def kron_rotate(x: np.ndarray, P1: np.ndarray, P2: np.ndarray) -> np.ndarray:
+    """x~ = x (P1 kron P2): float64 arithmetic, rounded once to float32."""
+    return kron_rotate_f64(x, P1, P2).astype(np.float32)
 
 
 def kron_rotate_dense(x: np.ndarray, P1: np.ndarray, P2: np.ndarray) -> np.ndarray:
@@ -201,16 +206,22 @@ class OracleLayer:
     """One shared quantized linear: folded + quantized weights, its P factors and LAS clips."""
 
     def __init__(self, W: np.ndarray, P1: np.ndarray, P2: np.ndarray, las: np.ndarray,
-                 a_bits: int, group: int = GROUP, fold: bool = True):
+                 a_bits: int, group: int = GROUP, fold: bool = True, Q1=None, Q2=None):
+        """Q1, Q2: the weight-side fold factors; by default P^{-T} rounded to
+        float32, the form in which a float32 library receives them."""
         self.P1 = np.asarray(P1, np.float32)
         self.P2 = np.asarray(P2, np.float32)
         self.las = np.asarray(las, np.float32)
         self.a_bits = a_bits
         self.group = group
         if fold:
-            Wt = fold_weights(W, inverse_transpose(self.P1), inverse_transpose(self.P2))
+            self.Q1 = inverse_transpose(self.P1).astype(np.float32) if Q1 is None else Q1
+            self.Q2 = inverse_transpose(self.P2).astype(np.float32) if Q2 is None else Q2
+            self.W_folded64 = kron_rotate_f64(W, self.Q1, self.Q2)
+            Wt = self.W_folded64.astype(np.float32)
         else:
             Wt = np.asarray(W, np.float32)
+            self.W_folded64 = Wt.astype(np.float64)
         self.W_folded = Wt
         self.qw, self.sw = quantize_weights(Wt, group)
         self.N, self.K = Wt.shape

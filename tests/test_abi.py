@@ -1,0 +1,121 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds, loads and
+exports every entry point include/lq.h declares, and argument validation
+rejects bad calls before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_ptq_looped_b200 import build as B
+from bit_ptq_looped_b200 import lq
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "lq.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lq_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return lq.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for want in ("lq_quantize_act", "lq_pack_weights", "lq_loop_linear", "lq_loop_stack"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+        assert name in lq.SIGNATURES, f"binding lacks {name}"
+
+
+def test_version(L):
+    assert L.lq_version() == 100
+
+
+def _err(L):
+    return L.lq_last_error().decode()
+
+
+def test_quantize_rejects_bad_arguments_before_launch(L):
+    fake = 1 << 20  # never dereferenced: every call below fails its checks first
+    # K not a multiple of 32
+    st = L.lq_quantize_act(fake, lq.LQ_F32, 4, 48, None, 0, None, 0, 1.0, 4, 32, fake, None,
+                           fake, None)
+    assert st == lq.LQ_ERR_SHAPE and "multiple of 32" in _err(L)
+    # unsupported bits / group
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, None, 0, None, 0, 1.0, 3, 32, fake, None,
+                             fake, None) == lq.LQ_ERR_UNSUPPORTED
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, None, 0, None, 0, 1.0, 4, 64, fake, None,
+                             fake, None) == lq.LQ_ERR_UNSUPPORTED
+    # non-positive LAS clip
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, None, 0, None, 0, 0.0, 4, 32, fake, None,
+                             fake, None) == lq.LQ_ERR_ARG
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, None, 0, None, 0, -1.0, 4, 32, fake, None,
+                             fake, None) == lq.LQ_ERR_ARG
+    # Kronecker sizes that do not multiply to K
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, fake, 4, fake, 8, 1.0, 4, 32, fake, None,
+                             fake, None) == lq.LQ_ERR_SHAPE
+    # only one factor
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, fake, 8, None, 0, 1.0, 4, 32, fake, None,
+                             fake, None) == lq.LQ_ERR_ARG
+    # factor sizes not multiples of 4
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 96, fake, 6, fake, 16, 1.0, 4, 32, fake, None,
+                             fake, None) == lq.LQ_ERR_UNSUPPORTED
+    # packed output with 8-bit codes
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, None, 0, None, 0, 1.0, 8, 32, None, fake,
+                             fake, None) == lq.LQ_ERR_UNSUPPORTED
+    # misaligned pointer
+    assert L.lq_quantize_act(fake + 4, lq.LQ_F32, 4, 64, None, 0, None, 0, 1.0, 4, 32, fake,
+                             None, fake, None) == lq.LQ_ERR_ALIGN
+    # unknown dtype, null outputs
+    assert L.lq_quantize_act(fake, 7, 4, 64, None, 0, None, 0, 1.0, 4, 32, fake, None, fake,
+                             None) == lq.LQ_ERR_UNSUPPORTED
+    assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, None, 0, None, 0, 1.0, 4, 32, None, None,
+                             fake, None) == lq.LQ_ERR_ARG
+
+
+def test_weight_entry_points_reject_bad_arguments(L):
+    fake = 1 << 20
+    h = ctypes.c_void_p()
+    assert L.lq_pack_weights(fake, 16, 48, 4, 32, ctypes.byref(h), None) == lq.LQ_ERR_SHAPE
+    assert L.lq_pack_weights(fake, 16, 64, 8, 32, ctypes.byref(h), None) == lq.LQ_ERR_UNSUPPORTED
+    assert L.lq_pack_weights(fake, 0, 64, 4, 32, ctypes.byref(h), None) == lq.LQ_ERR_ARG
+    assert L.lq_pack_weights(None, 16, 64, 4, 32, ctypes.byref(h), None) == lq.LQ_ERR_ARG
+    assert L.lq_pack_weights(fake, 16, 64, 4, 32, None, None) == lq.LQ_ERR_ARG
+    assert L.lq_quantize_weights(fake, 16, 64, 8, 32, fake, None, fake, None) == \
+        lq.LQ_ERR_UNSUPPORTED
+    # aliasing input and output
+    assert L.lq_fold_weights(fake, 16, 64, fake, 8, fake, 8, fake, None) == lq.LQ_ERR_ARG
+    assert L.lq_fold_weights(fake, 16, 64, fake, 4, fake, 8, fake + 16, None) == lq.LQ_ERR_SHAPE
+    las = (ctypes.c_float * 2)(1.0, 0.5)
+    assert L.lq_layer_create(None, fake, 4, fake, 4, las, 2, 4, ctypes.byref(h)) == lq.LQ_ERR_ARG
+
+
+def test_loop_entry_points_reject_bad_arguments(L):
+    fake = 1 << 20
+    assert L.lq_loop_linear(fake, lq.LQ_F32, 4, None, 0, fake, fake, 1 << 20, None) == \
+        lq.LQ_ERR_ARG
+    assert L.lq_loop_stack(fake, lq.LQ_F32, 4, None, 1, 4, lq.LQ_OPEN, fake, fake, 1 << 20,
+                           None) == lq.LQ_ERR_ARG
+    assert L.lq_workspace_bytes(None, 1, 4) == -1
+
+
+def test_inverse_transpose_host_helper():
+    rng = np.random.default_rng(0)
+    for n in (1, 4, 16, 88):
+        P = (rng.standard_normal((n, n)) + n * np.eye(n)).astype(np.float32)
+        got = lq.lq_inverse_transpose(P).numpy()
+        want = np.linalg.inv(P.astype(np.float64)).T
+        assert np.max(np.abs(got - want)) <= 1e-6 * max(1.0, np.max(np.abs(want)))
+    with pytest.raises(lq.LQError):
+        lq.lq_inverse_transpose(np.zeros((3, 3), np.float32))

@@ -1,0 +1,226 @@
+"""GPU parity of the quantized looped linear (lq_loop_linear, lq_loop_stack):
+tensor-core GEMM for prefill-sized M, weight-streaming GEMV for decode M."""
+import numpy as np
+import pytest
+import torch
+
+from bit_ptq_looped_b200 import lq, synth
+from oracle import lq_oracle as O
+from tests.parity import act_tensor, check_gemm, dev, host, linear_parity, weight_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def make_layer(mp, a_bits, T=None):
+    """Fold with the float32 P^{-T} factors and pack on the device; return
+    (lq Layer, oracle layer), with the weight-code near-tie differences in
+    ``layer.w_flips``."""
+    las = mp.las if T is None else mp.las[:T]
+    ol = O.OracleLayer(mp.W, mp.P1, mp.P2, las, a_bits)
+    Wf = lq.lq_fold_weights(dev(mp.W), dev(ol.Q1), dev(ol.Q2))
+    wq = lq.lq_pack_weights(Wf)
+    layer = lq.lq_layer_create(wq, dev(mp.P1), dev(mp.P2), las, a_bits)
+    c4, sc = lq.wq_tensors(wq)
+    layer.w_flips = weight_parity(host(c4), host(sc), ol)
+    return layer, ol
+
+
+def _integer_problem(M, N, K, a_bits, seed):
+    """Integer codes whose every group holds +-q_max: all steps are exactly 1."""
+    rng = np.random.default_rng(seed)
+    qmax = 7 if a_bits == 4 else 127
+    x = rng.integers(-qmax, qmax + 1, size=(M, K)).astype(np.float32)
+    w = rng.integers(-7, 8, size=(N, K)).astype(np.float32)
+    x[:, ::32] = qmax
+    w[:, 1::32] = -7
+    return x, w
+
+
+@pytest.mark.parametrize("a_bits", [4, 8])
+@pytest.mark.parametrize("MNK", [(128, 128, 128), (256, 384, 512), (200, 144, 2048),
+                                 (1000, 2048, 256), (33, 256, 128)])
+def test_gemm_exact_on_integer_problems(a_bits, MNK):
+    """With unit steps the library must return the exact integer product."""
+    M, N, K = MNK
+    a = 4 if K <= 512 else K // 128
+    b = K // a
+    x, w = _integer_problem(M, N, K, a_bits, seed=M + N + K)
+    wq = lq.lq_pack_weights(dev(w))
+    eye_a, eye_b = torch.eye(a, device="cuda"), torch.eye(b, device="cuda")
+    layer = lq.lq_layer_create(wq, eye_a, eye_b, [1.0], a_bits)
+    y = host(lq.lq_loop_linear(dev(x), layer, 0))
+    torch.cuda.synchronize()
+    want = x.astype(np.int64) @ w.astype(np.int64).T
+    np.testing.assert_array_equal(y, want.astype(np.float32))
+
+
+@pytest.mark.parametrize("a_bits", [4, 8])
+@pytest.mark.parametrize("wl", [synth.TINY, synth.ATTN_PROJ, synth.MLP], ids=lambda w: w.name)
+def test_loop_linear_prefill(wl, a_bits):
+    params = synth.module_params(wl)
+    for lin, mp in zip(wl.linears, params):
+        layer, ol = make_layer(mp, a_bits)
+        M = wl.M if wl.M <= 2048 else 2048
+        for t in range(wl.T):
+            x = synth.loop_input(wl, lin, t, rows=np.arange(M))
+            xd = act_tensor(x, wl.x_dtype)
+            y = lq.lq_loop_linear(xd, layer, t)
+            q8, _, s = lq.lq_quantize_act(xd, dev(mp.P1), dev(mp.P2), float(mp.las[t]), a_bits)
+            torch.cuda.synchronize()
+            linear_parity(host(y), x, ol, t, host(q8), host(s), layer.w_flips)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("N", [2048, 5632])
+@pytest.mark.parametrize("a_bits", [8, 4])
+def test_loop_linear_decode(M, N, a_bits):
+    wl = synth.decode_workload(M, N, a_bits)
+    (mp,) = synth.module_params(wl)
+    (lin,) = wl.linears
+    layer, ol = make_layer(mp, a_bits)
+    for t in range(wl.T):
+        x = synth.loop_input(wl, lin, t)
+        xd = act_tensor(x, wl.x_dtype)
+        y = lq.lq_loop_linear(xd, layer, t)
+        q8, _, s = lq.lq_quantize_act(xd, dev(mp.P1), dev(mp.P2), float(mp.las[t]), a_bits)
+        torch.cuda.synchronize()
+        linear_parity(host(y), x, ol, t, host(q8), host(s), layer.w_flips)
+
+
+@pytest.mark.parametrize("M", [0, 1, 17, 129, 300])
+def test_loop_linear_ragged_rows(M):
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    (lin,) = wl.linears
+    layer, ol = make_layer(mp, 4)
+    rng = np.random.default_rng(M)
+    x = rng.standard_normal((M, lin.K)).astype(np.float32)
+    y = lq.lq_loop_linear(dev(x), layer, 2)
+    torch.cuda.synchronize()
+    if M == 0:
+        assert y.numel() == 0
+        return
+    q8, _, s = lq.lq_quantize_act(dev(x), dev(mp.P1), dev(mp.P2), float(mp.las[2]), 4)
+    torch.cuda.synchronize()
+    linear_parity(host(y), x, ol, 2, host(q8), host(s), layer.w_flips)
+
+
+def test_loop_linear_rejects_bad_calls():
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    layer, _ = make_layer(mp, 4)
+    x = torch.zeros((64, 256), device="cuda")
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_loop_linear(x, layer, 4)
+    assert e.value.status == lq.LQ_ERR_SHAPE
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_loop_linear(x, layer, -1)
+    assert e.value.status == lq.LQ_ERR_SHAPE
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_loop_linear(x, layer, 0, ws=ws)
+    assert e.value.status == lq.LQ_ERR_WORKSPACE
+
+
+def _stack_inputs(wl, M):
+    xs = [[synth.loop_input(wl, lin, t, rows=np.arange(M)) for lin in wl.linears]
+          for t in range(wl.T)]
+    flat = np.concatenate([xs[t][l].ravel() for t in range(wl.T) for l in range(len(wl.linears))])
+    return xs, flat
+
+
+@pytest.mark.parametrize("wl,M", [(synth.TINY, 64), (synth.MLP, 384), (synth.ATTN_PROJ, 2048)],
+                         ids=["tiny", "mlp", "attn"])
+def test_loop_stack_open(wl, M):
+    params = synth.module_params(wl)
+    built = [make_layer(mp, wl.a_bits) for mp in params]
+    layers = [b[0] for b in built]
+    xs, flat = _stack_inputs(wl, M)
+    xd = act_tensor(flat, wl.x_dtype)
+    y1 = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M)
+    y2 = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, y=torch.empty_like(y1))
+    y3 = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, y=y1)  # graph replay, same args
+    torch.cuda.synchronize()
+    y1h = host(y1)
+    assert np.array_equal(y1h, host(y2)) and np.array_equal(y1h, host(y3))
+    off = 0
+    for t in range(wl.T):
+        for l, (lin, mp) in enumerate(zip(wl.linears, params)):
+            n = M * lin.N
+            yg = y1h[off:off + n].reshape(M, lin.N)
+            off += n
+            xd_tl = act_tensor(xs[t][l], wl.x_dtype)
+            q8, _, s = lq.lq_quantize_act(xd_tl, dev(mp.P1), dev(mp.P2), float(mp.las[t]),
+                                          wl.a_bits)
+            torch.cuda.synchronize()
+            linear_parity(yg, xs[t][l], built[l][1], t, host(q8), host(s), built[l][0].w_flips)
+
+
+def test_loop_stack_chain_tiny():
+    """Chain mode feeds y_{t} back as x_{t+1} (T = 4 loops of one shared layer)."""
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    (lin,) = wl.linears
+    layer, ol = make_layer(mp, 4)
+    x0 = synth.loop_input(wl, lin, 0)
+    y = host(lq.lq_loop_stack(dev(x0), [layer], wl.T, lq.LQ_CHAIN, M=wl.M))
+    torch.cuda.synchronize()
+    ys = O.loop_stack_chain(x0, [ol], wl.T)
+    for t in range(wl.T):
+        check_gemm(y[t * wl.M * lin.N:(t + 1) * wl.M * lin.N].reshape(wl.M, lin.N), ys[t][0],
+                   what=f"chain t={t}")
+
+
+def test_loop_stack_chain_shape_check():
+    wl = synth.MLP
+    params = synth.module_params(wl)
+    layers = [make_layer(mp, 4)[0] for mp in params[:2]]  # gate -> up: 5632 != 2048
+    x = torch.zeros((64, 2048), device="cuda")
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_loop_stack(x, layers, 2, lq.LQ_CHAIN, M=64)
+    assert e.value.status == lq.LQ_ERR_SHAPE
+
+
+def test_loop_stack_inside_caller_capture():
+    """When the caller's stream is capturing, the stack records into that capture."""
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    layer, _ = make_layer(mp, 4)
+    xs, flat = _stack_inputs(wl, wl.M)
+    xd = act_tensor(flat, wl.x_dtype)
+    ref = lq.lq_loop_stack(xd, [layer], wl.T, lq.LQ_OPEN, M=wl.M)
+    y = torch.zeros_like(ref)
+    ws = lq.workspace([layer], wl.M)
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        lq.lq_loop_stack(xd, [layer], wl.T, lq.LQ_OPEN, M=wl.M, y=y, ws=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+
+
+def test_calib_block_full_size_sampled_rows():
+    """Full 262144-token calibration block: every (module, loop) at full size,
+    checked on sampled rows (rows are independent)."""
+    wl = synth.CALIB_BLOCK
+    params = synth.module_params(wl)
+    rng = np.random.default_rng(5)
+    rows = np.sort(rng.choice(wl.M, 192, replace=False))
+    rows[0], rows[-1] = 0, wl.M - 1
+    rows_d = torch.from_numpy(rows).cuda()
+    for l, (lin, mp) in enumerate(zip(wl.linears, params)):
+        layer, ol = make_layer(mp, wl.a_bits)
+        for t in ((0, 3) if l % 2 else (1, 2)):
+            x = synth.device_loop_input(wl, lin, t)
+            y = lq.lq_loop_linear(x, layer, t)
+            ys = host(y[rows_d])
+            xs = x[rows_d].float().cpu().numpy()
+            del y
+            q8, _, s = lq.lq_quantize_act(x[rows_d].contiguous(), dev(mp.P1), dev(mp.P2),
+                                          float(mp.las[t]), wl.a_bits)
+            torch.cuda.synchronize()
+            linear_parity(ys, xs, ol, t, host(q8), host(s), layer.w_flips)
+            del x
+        lq.lq_check_device()

@@ -1,0 +1,145 @@
+"""GPU parity of the quantizers (lq_quantize_act, lq_quantize_weights,
+lq_pack_weights, lq_fold_weights) against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+from bit_ptq_looped_b200 import lq, synth
+from oracle import lq_oracle as O
+from tests.parity import act_tensor, check_codes_near_tie, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _outlier_matrix(M, K, seed, frac=0.02, mult=20.0, scale=1.0):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((M, K)) * scale).astype(np.float32)
+    ch = rng.choice(K, max(1, int(round(frac * K))), replace=False)
+    x[:, ch] *= np.float32(mult)
+    return x
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("x_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("c", [1.0, 0.7, 0.8374])
+@pytest.mark.parametrize("shape", [(1, 32), (3, 64), (257, 256), (2048, 2048), (130, 5632)])
+def test_quantize_only_bit_exact(bits, x_dtype, c, shape):
+    M, K = shape
+    x = _outlier_matrix(M, K, seed=M * 7 + K)
+    if x_dtype == "bf16":
+        x = synth.round_bf16(x)
+    x[0, :32] = 0.0  # one all-zero group
+    if M > 2:
+        x[2, 32:64] = np.float32(3.5) * np.sign(x[2, 32:64])  # many exact ties
+    q8, q4, s = lq.lq_quantize_act(act_tensor(x, x_dtype), None, None, c, bits,
+                                   want_codes4=(bits == 4))
+    torch.cuda.synchronize()
+    q_or, s_or = O.quantize_groups(x, c, bits)
+    np.testing.assert_array_equal(host(s), s_or)
+    np.testing.assert_array_equal(host(q8), q_or)
+    if bits == 4:
+        np.testing.assert_array_equal(host(q4), O.pack_int4(q_or))
+
+
+def test_quantize_only_edge_values():
+    # powers of two, subnormal-range values and exact half-way ratios
+    K = 64
+    rows = [np.full(K, 7.0), np.linspace(-7, 7, K), np.full(K, 1e-39),
+            np.concatenate([[2.0 ** -120], np.zeros(K - 1)]),
+            np.arange(K) * 0.5 - 16, np.full(K, -3.0e37)]
+    x = np.stack(rows).astype(np.float32)
+    for bits in (4, 8):
+        for c in (1.0, 0.75, 1.5):
+            q8, _, s = lq.lq_quantize_act(dev(x), None, None, c, bits)
+            torch.cuda.synchronize()
+            q_or, s_or = O.quantize_groups(x, c, bits)
+            np.testing.assert_array_equal(host(s), s_or)
+            np.testing.assert_array_equal(host(q8), q_or)
+
+
+def test_quantize_empty_input_is_a_noop():
+    x = torch.empty((0, 64), dtype=torch.float32, device="cuda")
+    q8, _, s = lq.lq_quantize_act(x, None, None, 1.0, 4)
+    torch.cuda.synchronize()
+    assert q8.numel() == 0 and s.numel() == 0
+
+
+WORKLOADS = [synth.TINY, synth.ATTN_PROJ, synth.MLP]
+
+
+@pytest.mark.parametrize("wl", WORKLOADS, ids=lambda w: w.name)
+@pytest.mark.parametrize("bits", [4, 8])
+def test_fused_rotate_quantize(wl, bits):
+    params = synth.module_params(wl)
+    for l, (lin, mp) in enumerate(zip(wl.linears, params)):
+        M = min(wl.M, 512) + (3 if wl.M > 64 else 0)  # several row tiles and a ragged tail
+        for t in (0, wl.T - 1):
+            x = synth.loop_input(wl, lin, t, rows=np.arange(M))
+            c = float(mp.las[t])
+            q8, q4, s = lq.lq_quantize_act(act_tensor(x, wl.x_dtype), dev(mp.P1), dev(mp.P2), c,
+                                           bits, want_codes4=(bits == 4))
+            torch.cuda.synchronize()
+            xt64 = O.kron_rotate_f64(x, mp.P1, mp.P2)
+            q_or, s_or = O.quantize_groups(xt64.astype(np.float32), c, bits)
+            flips = check_codes_near_tie(host(q8), host(s), q_or, s_or, xt64)
+            if bits == 4:
+                np.testing.assert_array_equal(O.unpack_int4(host(q4)), host(q8))
+            # the float64 rotation rounds like the oracle's: no differences expected here
+            assert len(flips) == 0
+
+
+def test_fused_rotation_identity_factors_reduce_to_plain_rtn():
+    M, K = 100, 2048
+    x = _outlier_matrix(M, K, seed=3)
+    eye1, eye2 = np.eye(32, dtype=np.float32), np.eye(64, dtype=np.float32)
+    q8, _, s = lq.lq_quantize_act(dev(x), dev(eye1), dev(eye2), 0.9, 4)
+    torch.cuda.synchronize()
+    q_or, s_or = O.quantize_groups(x, 0.9, 4)
+    np.testing.assert_array_equal(host(s), s_or)
+    np.testing.assert_array_equal(host(q8), q_or)
+
+
+def test_weight_quantize_and_pack_bit_exact():
+    wl = synth.MLP
+    for mp in synth.module_params(wl):
+        W = mp.W
+        Wt = O.fold_weights(W, O.inverse_transpose(mp.P1), O.inverse_transpose(mp.P2))
+        q8, q4, s = lq.lq_quantize_weights(dev(Wt))
+        torch.cuda.synchronize()
+        q_or, s_or = O.quantize_weights(Wt)
+        np.testing.assert_array_equal(host(s), s_or)
+        np.testing.assert_array_equal(host(q8), q_or)
+        np.testing.assert_array_equal(host(q4), O.pack_int4(q_or))
+        wq = lq.lq_pack_weights(dev(Wt))
+        c4, sc = lq.wq_tensors(wq)
+        np.testing.assert_array_equal(host(c4), O.pack_int4(q_or))
+        np.testing.assert_array_equal(host(sc), s_or)
+        info = wq.info()
+        assert info["N"] == W.shape[0] and info["K"] == W.shape[1]
+        wq.free()
+
+
+@pytest.mark.parametrize("ab", [(16, 16), (32, 64), (64, 88)])
+def test_fold_weights(ab):
+    a, b = ab
+    rng = np.random.default_rng(a * b)
+    N = 300
+    W = (rng.standard_normal((N, a * b)) * 0.02).astype(np.float32)
+    P1 = synth.orthogonal(a, 1, 0, 1)
+    P2 = synth.orthogonal(b, 1, 0, 2)
+    Q1 = O.inverse_transpose(P1).astype(np.float32)
+    Q2 = O.inverse_transpose(P2).astype(np.float32)
+    got = host(lq.lq_fold_weights(dev(W), dev(Q1), dev(Q2)))
+    torch.cuda.synchronize()
+    want64 = O.kron_rotate_f64(W, Q1, Q2)
+    want = want64.astype(np.float32)
+    # float64 sums in a different order round to the same float32 except
+    # within float64 rounding of a float32 rounding boundary
+    ulp = np.spacing(np.abs(want))
+    assert np.all(np.abs(got - want) <= ulp)
+    assert (got != want).mean() < 1e-4
+    # and W~ stays an exact-arithmetic fold: x W^T = (x P)(W~)^T up to float rounding
+    x = rng.standard_normal((4, a * b))
+    lhs = x @ W.astype(np.float64).T
+    rhs = (x @ np.kron(P1.astype(np.float64), P2.astype(np.float64))) @ got.astype(np.float64).T
+    assert np.max(np.abs(lhs - rhs)) <= 1e-5 * np.max(np.abs(lhs))
