@@ -760,3 +760,41 @@ lq_status lq_check_device(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// helpers for lq_loop_linear_noalloc (lq_noalloc.cu): the same checks and the
+// same kernels as lq_loop_linear, with the workspace supplied by the caller
+// of these helpers
+// ---------------------------------------------------------------------------
+namespace lq {
+
+lq_status noalloc_check(const void* d_x, int32_t x_dtype, int64_t M, const lq_layer* layer,
+                        int32_t t, float* d_y) {
+  lq_status st;
+  if ((st = check_layer_call(layer, M, x_dtype)) != LQ_OK) return st;
+  if (t < 0 || t >= layer->T) {
+    set_error("loop index t=%d outside [0, %d)", t, layer->T);
+    return LQ_ERR_SHAPE;
+  }
+  if (M == 0) return LQ_OK;
+  if (!d_x || !d_y) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_x) || !aligned16(d_y)) {
+    set_error("x and y must be 16-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  return LQ_OK;
+}
+
+int64_t noalloc_ws_bytes(const lq_layer* layer, int64_t M) {
+  return ws_bytes_for(M, layer->wq->K);
+}
+
+lq_status noalloc_enqueue(const void* d_x, int32_t x_dtype, int64_t M, const lq_layer* layer,
+                          int32_t t, float* d_y, void* d_ws, cudaStream_t s) {
+  return enqueue_linear(d_x, x_dtype, M, layer, t, d_y, d_ws, s);
+}
+
+}  // namespace lq

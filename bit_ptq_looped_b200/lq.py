@@ -48,6 +48,7 @@ SIGNATURES = {
     "lq_loop_linear": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
     "lq_check_device": (_i32, [_vp]),
+    "lq_loop_linear_noalloc": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp]),
     "lq_probe_enable": (_i32, [_i32]),
     "lq_probe_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]),
 }
@@ -297,6 +298,22 @@ def lq_loop_stack(x: torch.Tensor, layers: Sequence[Layer], T: int, mode: int = 
     st = lib().lq_loop_stack(_dev(x, "x"), dt, M, p, len(layers), T, mode, _dev(y, "y"),
                              _dev(ws, "ws"), ws.numel(), _stream(stream))
     _check(st, "lq_loop_stack")
+    return y
+
+
+LQ_NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def lq_loop_linear_noalloc(x: torch.Tensor, layer: Layer, t: int, *,
+                           y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """lq_loop_linear without a workspace (the library's fixed scratch is used;
+    see include/lq.h).  ``y`` must be given by callers that cannot allocate."""
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, layer.N), dtype=torch.float32, device=x.device)
+    st = lib().lq_loop_linear_noalloc(_dev(x, "x"), _dtype_code(x), M, layer.handle, t,
+                                      _dev(y, "y"), _stream(stream))
+    _check(st, "lq_loop_linear_noalloc")
     return y
 
 

@@ -195,6 +195,34 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
                         float* d_y, void* d_ws, int64_t ws_bytes, void* stream);
 
 /*
+ * lq_loop_linear_noalloc -- lq_loop_linear for callers that cannot allocate
+ * device memory, so cannot provide its workspace: for instance the enqueue
+ * hook of another runtime that hands over only input and output buffers, a
+ * serving loop that forbids allocation once it has started, or code running
+ * while another framework's caching allocator owns all free device memory.
+ * (The paper has no counterpart; this is a deployment convenience.)
+ *
+ * Same arguments, checks, kernels and results as lq_loop_linear, minus the
+ * workspace.  The scratch is a fixed device array of LQ_NOALLOC_SCRATCH_BYTES
+ * built into the library; every GPU that loads the library holds it until the
+ * process exits.  The call allocates nothing (no cudaMalloc, no cudaFree).
+ *   - Calls needing more scratch than that, lq_workspace_bytes(&layer, 1, M)
+ *     > LQ_NOALLOC_SCRATCH_BYTES (about M*K*(1 + 1/8) bytes), fail with
+ *     LQ_ERR_WORKSPACE and enqueue nothing.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Each call writes every scratch byte it reads before reading it, so
+ *     nothing has to start at zero; but calls whose work overlaps on the GPU
+ *     (for instance on two streams without ordering between them) race on the
+ *     array and give wrong results.
+ *   - The first call on a device looks the array's device address up (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ */
+#define LQ_NOALLOC_SCRATCH_BYTES (16ll << 20)
+lq_status lq_loop_linear_noalloc(const void* d_x, int32_t x_dtype, int64_t M,
+                                 const lq_layer* layer, int32_t t, float* d_y, void* stream);
+
+/*
  * Kernel timing probe.  While enabled (on != 0), lq_loop_linear and
  * lq_loop_stack launch their kernels directly (no graph) and bracket each one
  * with CUDA events recorded on the launching stream.  lq_probe_read waits for
