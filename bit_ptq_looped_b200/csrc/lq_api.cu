@@ -93,8 +93,9 @@ lq_status check_kron(int64_t K, const float* P1, int a, const float* P2, int b, 
     set_error("a*b = %d*%d != K = %lld", a, b, (long long)K);
     return LQ_ERR_SHAPE;
   }
-  if (a % 4 || b % 4 || a > 128 || b > 128) {
-    set_error("Kronecker factor sizes must be multiples of 4 and at most 128 (a=%d, b=%d)", a, b);
+  if (a % 16 || b % 8 || a > 128 || b > 128) {
+    set_error("Kronecker factor sizes must be a multiple of 16 (a) and of 8 (b), at most 128 "
+              "(a=%d, b=%d)", a, b);
     return LQ_ERR_UNSUPPORTED;
   }
   if (rotate_smem_bytes(a, b, nullptr) == 0) {

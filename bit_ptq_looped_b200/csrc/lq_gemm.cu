@@ -19,8 +19,12 @@
 //         integer group sum (|acc| <= 32*49) exactly;
 //   W4A8: codes stored as int8 and multiplied with kind::i8 (int32 sums).
 //
-// Warp roles (320 threads): warps 0-7 epilogue (warp w reads TMEM lane
-// quadrant w % 4, column half w / 4), warp 8 TMA producer, warp 9 MMA issuer.
+// Warp roles (576 threads): warps 0-15 epilogue, warp 16 TMA producer, warp
+// 17 MMA issuer.  Epilogue warp w reads TMEM lane quadrant w % 4 (its 32 rows)
+// and the 32-column block w / 4 of every group's accumulator with one load,
+// releases the buffer, and folds the columns with packed f32x2 arithmetic.
+// (Variants that pipelined the TMEM loads across pieces or groups, split the
+// groups between two warp sets, or ran two CTAs per SM measured no faster.)
 // Every mbarrier wait is bounded; on expiry the kernel records
 // LQ_ERR_DEVICE_TIMEOUT in a device status word, stops all roles, frees its
 // TMEM and returns.
@@ -40,11 +44,11 @@ constexpr int GPS = BK / kGroup;        // groups per stage = 4
 constexpr int STAGES = 5;
 constexpr int ACC_BUFS = 4;             // 4 x 128 TMEM columns
 constexpr int TMEM_COLS = 512;
-constexpr int EPI_WARPS = 8;
-constexpr int WARP_TMA = 8;
-constexpr int WARP_MMA = 9;
-constexpr int THREADS = 320;
-constexpr int EPI_COLS = BN / 2;        // columns per epilogue warp
+constexpr int EPI_WARPS = 16;          // 4 lane quadrants x 4 column blocks
+constexpr int WARP_TMA = EPI_WARPS;
+constexpr int WARP_MMA = EPI_WARPS + 1;
+constexpr int THREADS = 32 * (EPI_WARPS + 2);
+constexpr int EPI_COLS = BN * 4 / EPI_WARPS;  // 32 columns per epilogue warp
 
 constexpr uint32_t A_BYTES = BM * BK;          // 16 KB
 constexpr uint32_t B_BYTES = BN * BK;          // 16 KB
@@ -98,14 +102,16 @@ __host__ __device__ constexpr uint32_t instr_desc() {
          | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
+// two accumulator columns as float32: E4M3 path reads float32 sums directly;
+// int8 path converts exactly (|acc| < 2^22) through the mantissa of 1.5 * 2^23
 template <int kKindI8>
-__device__ __forceinline__ float acc_to_f32(uint32_t r) {
+__device__ __forceinline__ float2 acc_pair(uint32_t r0, uint32_t r1) {
   if (kKindI8) {
-    // exact int32 -> float32 for |acc| < 2^22: place it in the mantissa of 1.5 * 2^23
-    return __int_as_float((int)r + 0x4B400000) - 12582912.0f;
-  } else {
-    return __uint_as_float(r);
+    const float2 biased = make_float2(__int_as_float((int)r0 + 0x4B400000),
+                                      __int_as_float((int)r1 + 0x4B400000));
+    return fadd2(biased, make_float2(-12582912.0f, -12582912.0f));
   }
+  return make_float2(__uint_as_float(r0), __uint_as_float(r1));
 }
 
 template <int kKindI8>
@@ -218,71 +224,49 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_wait_drain(bar_drain, 0u);
     }
   } else {
-    // ---------------- epilogue: warps 0..7 ----------------
+    // ---------------- epilogue: warps 0..EPI_WARPS-1 ----------------
+    static_assert(EPI_COLS == 32, "one 32-column TMEM load per group");
     const int quad = warp & 3;
     const int col0 = (warp >> 2) * EPI_COLS;
     const int row = quad * 32 + lane;
-    float acc[EPI_COLS];
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)col0;
+    float2 acc[EPI_COLS / 2];
 #pragma unroll
-    for (int i = 0; i < EPI_COLS; ++i) acc[i] = 0.f;
-    int gi = 0;
+    for (int i = 0; i < EPI_COLS / 2; ++i) acc[i] = make_float2(0.f, 0.f);
     bool ok = true;
-    for (int kb = 0; kb < n_kb && ok; ++kb) {
-      const int st = kb % STAGES;
-      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-      if (!mbar_wait_bounded(bar_full + 8 * st, ph, abort_flag, &g_gemm_status, kWaitLimitNs)) {
-        ok = false;
-        break;
-      }
-      const float4 sa4 =
-          *reinterpret_cast<const float4*>(gbase + OFF_SA + st * SA_BYTES + row * 16);
-      const float sa[GPS] = {sa4.x, sa4.y, sa4.z, sa4.w};
-      const float* sw_st = reinterpret_cast<const float*>(gbase + OFF_SW + st * SW_BYTES);
-#pragma unroll
-      for (int j = 0; j < GPS; ++j, ++gi) {
-        const int buf = gi % ACC_BUFS;
-        const uint32_t aph = (uint32_t)(gi / ACC_BUFS) & 1u;
-        if (!mbar_wait_bounded(bar_accf + 8 * buf, aph, abort_flag, &g_gemm_status,
-                               kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t r0[32], r1[32];
-        const uint32_t taddr =
-            tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN + col0);
-        tmem_ld_32x32b_x32(taddr, r0);
-        tmem_ld_32x32b_x32(taddr + 32u, r1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
-        const float s = sa[j];
-        const float4* swv = reinterpret_cast<const float4*>(sw_st + j * BN + col0);
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 w = swv[c4];
-          acc[4 * c4 + 0] = fmaf(s * w.x, acc_to_f32<kKindI8>(r0[4 * c4 + 0]), acc[4 * c4 + 0]);
-          acc[4 * c4 + 1] = fmaf(s * w.y, acc_to_f32<kKindI8>(r0[4 * c4 + 1]), acc[4 * c4 + 1]);
-          acc[4 * c4 + 2] = fmaf(s * w.z, acc_to_f32<kKindI8>(r0[4 * c4 + 2]), acc[4 * c4 + 2]);
-          acc[4 * c4 + 3] = fmaf(s * w.w, acc_to_f32<kKindI8>(r0[4 * c4 + 3]), acc[4 * c4 + 3]);
-        }
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 w = swv[8 + c4];
-          acc[32 + 4 * c4 + 0] =
-              fmaf(s * w.x, acc_to_f32<kKindI8>(r1[4 * c4 + 0]), acc[32 + 4 * c4 + 0]);
-          acc[32 + 4 * c4 + 1] =
-              fmaf(s * w.y, acc_to_f32<kKindI8>(r1[4 * c4 + 1]), acc[32 + 4 * c4 + 1]);
-          acc[32 + 4 * c4 + 2] =
-              fmaf(s * w.z, acc_to_f32<kKindI8>(r1[4 * c4 + 2]), acc[32 + 4 * c4 + 2]);
-          acc[32 + 4 * c4 + 3] =
-              fmaf(s * w.w, acc_to_f32<kKindI8>(r1[4 * c4 + 3]), acc[32 + 4 * c4 + 3]);
-        }
-      }
+    for (int gi = 0; gi < G && ok; ++gi) {
+      const int kb = gi / GPS, j = gi % GPS, st = kb % STAGES;
+      if (j == 0)  // the group's steps arrive with its stage
+        ok = mbar_wait_bounded(bar_full + 8 * st, (uint32_t)(kb / STAGES) & 1u, abort_flag,
+                               &g_gemm_status, kWaitLimitNs);
+      const int buf = gi % ACC_BUFS;
+      ok = ok && mbar_wait_bounded(bar_accf + 8 * buf, (uint32_t)(gi / ACC_BUFS) & 1u,
+                                   abort_flag, &g_gemm_status, kWaitLimitNs);
       if (!ok) break;
+      tc_fence_after();
+      uint32_t r[EPI_COLS];
+      tmem_ld_32x32b_x32(lane_base + (uint32_t)(buf * BN), r);
+      tmem_wait_ld();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty + 8 * st);
+      if (lane == 0) mbar_arrive(bar_acce + 8 * buf);  // accumulator buffer is free again
+      const float s_a =
+          reinterpret_cast<const float*>(gbase + OFF_SA + st * SA_BYTES + row * 16)[j];
+      const float2 s2 = make_float2(s_a, s_a);
+      const float4* swv =
+          reinterpret_cast<const float4*>(gbase + OFF_SW + st * SW_BYTES) + (j * BN + col0) / 4;
+#pragma unroll
+      for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
+        const float4 w = swv[c4];
+        acc[2 * c4] = ffma2(fmul2(s2, make_float2(w.x, w.y)),
+                            acc_pair<kKindI8>(r[4 * c4 + 0], r[4 * c4 + 1]), acc[2 * c4]);
+        acc[2 * c4 + 1] = ffma2(fmul2(s2, make_float2(w.z, w.w)),
+                                acc_pair<kKindI8>(r[4 * c4 + 2], r[4 * c4 + 3]), acc[2 * c4 + 1]);
+      }
+      if (j == GPS - 1) {  // this stage's shared-memory steps are no longer needed
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty + 8 * st);
+      }
     }
     const int gm = m0 + row;
     if (ok && gm < M) {
@@ -291,7 +275,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
         if (n0 + col0 + 4 * c4 < N)
           *reinterpret_cast<float4*>(yr + 4 * c4) =
-              make_float4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
+              make_float4(acc[2 * c4].x, acc[2 * c4].y, acc[2 * c4 + 1].x, acc[2 * c4 + 1].y);
       }
     }
   }

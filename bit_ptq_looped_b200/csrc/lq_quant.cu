@@ -49,6 +49,14 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* __restrict__ x, int64
 
 // Quantize the 8 values a thread holds; the 4 consecutive lanes 4j..4j+3 of
 // a warp hold one group of 32.  Every lane of the warp must call this.
+//
+// The code is rne(fl32(x / s)), decided without a division per element:
+// r1 = fl32(x * fl32(1 / s)) lies within 1.5 ulp of fl32(x / s), so the two
+// round to the same integer unless a half-integer lies within that distance
+// of r1.  Values within 2^-14 of a half-integer (far more than 1.5 ulp for
+// every |r1| < 128, the range that can round inside [-q_max, q_max]) take the
+// true IEEE division instead; NaN or infinite r1 (s so small that 1 / s
+// overflows) fails the same test and takes it too.
 __device__ __forceinline__ float quant_group8(const float (&v)[8], float c, int qmax,
                                               int (&q)[8]) {
   float am = 0.f;
@@ -58,18 +66,30 @@ __device__ __forceinline__ float quant_group8(const float (&v)[8], float c, int 
   am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
   // s = fl32(fl32(c * absmax) / q_max): two IEEE round-to-nearest operations
   const float s = __fdiv_rn(__fmul_rn(c, am), (float)qmax);
+  const float inv = __frcp_rn(s);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     int qi = 0;
     if (s != 0.f) {
-      const float r = __fdiv_rn(v[i], s);  // fl32(x / s), true division
-      qi = __float2int_rn(r);              // round half to even
-      qi = min(max(qi, -qmax), qmax);
+      const float r1 = __fmul_rn(v[i], inv);
+      const float rr = rintf(r1);
+      const float tie_dist = 0.5f - fabsf(r1 - rr);
+      float r = rr;
+      if (!(tie_dist > 6.103515625e-05f))  // 2^-14, or NaN
+        r = rintf(__fdiv_rn(v[i], s));     // fl32(x / s), true division, then RNE
+      qi = (int)fminf(fmaxf(r, (float)-qmax), (float)qmax);
     }
     q[i] = qi;
   }
   return s;
 }
+
+// floor(n / d) for n, d < 2^16 with one multiply-high (d fixed per launch)
+struct FastDiv {
+  uint32_t d, m;
+  __device__ __forceinline__ explicit FastDiv(uint32_t dd) : d(dd), m((0xFFFFFFFFu / dd) + 1u) {}
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return d == 1u ? n : __umulhi(n, m); }
+};
 
 // Write one thread's 8 codes (and its group's step from lane 4j).
 __device__ __forceinline__ void store_codes(const int (&q)[8], float s, int64_t chunk,
@@ -124,30 +144,94 @@ __global__ void __launch_bounds__(kThreads) k_quant_only(const Tin* __restrict__
 
 // ---------------------------------------------------------------------------
 // fused Kronecker rotation + quantization
+//
+// A block takes R token rows.  Stage 1 forms Y = X P2 for the R*a rows of
+// the row-major reshapes X (a x b each); stage 2 forms Z_r = P1^T Y_r per
+// token.  Both stages run on the FP64 tensor-core MMA (m8n8k4, float64
+// inputs, products and sums), so x~ is the float64 value rounded once to
+// float32.  Shared-memory operands are stored so that every fragment load
+// reads 8 rows x 4 consecutive doubles of a row-major array whose row pitch
+// is the row length + 4 doubles (conflict-free):
+//   P2T[j][q] = P2[q][j]   (b x (b+4))      YT[r][j][p] = Y[r][p][j]  (R*b x (a+4))
+//   P1T[i][p] = P1[p][i]   (a x (a+4))
+//   X[(r,i)][q] float32 (exact copies of the bf16/fp32 inputs; (R*a) x (b+4)),
+//   Z[r][i][j] float32 with the same pitch, aliased on X once stage 1 is done.
 // ---------------------------------------------------------------------------
-struct RotSmem {
-  double* P1;  // a x a
-  double* P2;  // b x b
-  double* X;   // R x K   (input rows, then the float32 result Z aliased on it)
-  double* Y;   // R x K   (X P2)
+struct RotLayout {
+  int a, b, R, lda, ldb, ldz;
+  size_t off_p1t, off_yt, off_x, bytes;  // double offsets (X: float offset base) / bytes
 };
 
-__device__ __forceinline__ void load_row_chunk(const float* __restrict__ x, int64_t chunk,
-                                               double* dst) {
+__host__ __device__ inline RotLayout rot_layout(int a, int b, int R) {
+  RotLayout L;
+  L.a = a;
+  L.b = b;
+  L.R = R;
+  L.lda = a + 4;
+  L.ldb = b + 4;
+  L.ldz = b + 4;
+  L.off_p1t = (size_t)b * L.ldb;  // after P2T (doubles)
+  L.off_yt = L.off_p1t + (size_t)a * L.lda;
+  L.off_x = L.off_yt + (size_t)R * b * L.lda;  // doubles before the float region
+  L.bytes = 8 * L.off_x + 4 * (size_t)R * a * L.ldb;
+  return L;
+}
+
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
+// One warp task of an (8*TM) x (8*TN) output block of C = A B, with A given
+// row-major (A[row][k], pitch lda_) and B given transposed (Bt[col][k], pitch
+// ldb_).  Output tiles beyond n_col_tiles are skipped.  Calls
+// emit(row, col, v0, v1) for C[row][col], C[row][col + 1].
+template <int TM, int TN, typename TA, typename Emit>
+__device__ __forceinline__ void warp_mma_task(const TA* __restrict__ A, int lda_,
+                                              const double* __restrict__ Bt, int ldb_, int kdim,
+                                              int row0, int col_tile0, int n_col_tiles,
+                                              Emit emit) {
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  double acc[TM][TN][2];
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+  const TA* a_ptr = A + (size_t)(row0 + g) * lda_ + t;
+  const double* b_ptr = Bt + (size_t)(col_tile0 * 8 + g) * ldb_ + t;
+  for (int k = 0; k < kdim; k += 4) {
+    double av[TM], bv[TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i) av[i] = (double)a_ptr[(size_t)(8 * i) * lda_ + k];
+#pragma unroll
+    for (int j = 0; j < TN; ++j)
+      bv[j] = (col_tile0 + j < n_col_tiles) ? b_ptr[(size_t)(8 * j) * ldb_ + k] : 0.0;
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) dmma_8x8x4(acc[i][j], av[i], bv[j]);
+  }
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j)
+      if (col_tile0 + j < n_col_tiles)
+        emit(row0 + 8 * i + g, (col_tile0 + j) * 8 + 2 * t, acc[i][j][0], acc[i][j][1]);
+}
+
+template <typename Tin>
+__device__ __forceinline__ void load_row_chunk8(const Tin* __restrict__ x, int64_t chunk,
+                                                float* dst) {
   float v[8];
   load8(x, chunk, v);
-  double2* d = reinterpret_cast<double2*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) d[i] = make_double2((double)v[2 * i], (double)v[2 * i + 1]);
+  float4* d = reinterpret_cast<float4*>(dst);
+  d[0] = make_float4(v[0], v[1], v[2], v[3]);
+  d[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
-__device__ __forceinline__ void load_row_chunk(const __nv_bfloat16* __restrict__ x,
-                                               int64_t chunk, double* dst) {
-  float v[8];
-  load8(x, chunk, v);
-  double2* d = reinterpret_cast<double2*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) d[i] = make_double2((double)v[2 * i], (double)v[2 * i + 1]);
-}
+
+constexpr int kRotTM = 2, kRotTN = 4;  // warp task: 16 x 32 outputs
 
 template <typename Tin, bool kStoreF32>
 __global__ void __launch_bounds__(kThreads) k_rotate_quant(
@@ -156,115 +240,107 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
     int opf, uint8_t* __restrict__ codes4, float* __restrict__ scales,
     float* __restrict__ out_f32) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  RotSmem sm;
-  sm.P1 = reinterpret_cast<double*>(smem_raw);
-  sm.P2 = sm.P1 + a * a;
-  sm.X = sm.P2 + b * b;
-  sm.Y = sm.X + (size_t)R * K;
-  float* Z = reinterpret_cast<float*>(sm.X);
+  const RotLayout L = rot_layout(a, b, R);
+  double* sm = reinterpret_cast<double*>(smem_raw);
+  double* P2T = sm;
+  double* P1T = sm + L.off_p1t;
+  double* YT = sm + L.off_yt;
+  float* X = reinterpret_cast<float*>(sm + L.off_x);
+  float* Z = X;  // (R*a) rows of pitch ldz floats, written after stage 1
 
-  const int tid = threadIdx.x;
-  for (int i = tid; i < a * a; i += kThreads) sm.P1[i] = (double)P1[i];
-  for (int i = tid; i < b * b; i += kThreads) sm.P2[i] = (double)P2[i];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  constexpr int kWarps = kThreads / 32;
+  for (int e = tid; e < b * b; e += kThreads) {
+    const int q = e / b, j = e - q * b;
+    P2T[(size_t)j * L.ldb + q] = (double)P2[e];
+  }
+  for (int e = tid; e < a * a; e += kThreads) {
+    const int p = e / a, i = e - p * a;
+    P1T[(size_t)i * L.lda + p] = (double)P1[e];
+  }
 
-  const int ct_n = b >> 2;           // column tiles (strided columns ct + jj*ct_n)
-  const int rt_n = (R * a) >> 2;     // row tiles of 4 rows of the R*a x b stacks
-  const int n_tiles = rt_n * ct_n;
-  const int row_chunks = K >> 3;     // 8-element chunks per token row
+  const int row_chunks = K >> 3;
+  const FastDiv fd_rowc((uint32_t)row_chunks), fd_b((uint32_t)b), fd_a((uint32_t)a);
+  // stage 1 tasks: (R*a/16) row pairs x ceil(b/32) column quads
+  const int ct = b >> 3;
+  const int s1_rt = (R * a) / (8 * kRotTM);
+  const int s1_ctq = (ct + kRotTN - 1) / kRotTN;
+  const int s1_tasks = s1_rt * s1_ctq;
+  // stage 2 tasks per token: (a/16) x ceil(b/32)
+  const int s2_rt = a / (8 * kRotTM);
+  const int s2_tasks = R * s2_rt * s1_ctq;
+  const FastDiv fd_s1ctq((uint32_t)s1_ctq), fd_s2tok((uint32_t)(s2_rt * s1_ctq));
 
   for (int64_t m0 = (int64_t)blockIdx.x * R; m0 < M; m0 += (int64_t)gridDim.x * R) {
     const int rows = (M - m0 < (int64_t)R) ? (int)(M - m0) : R;
-    __syncthreads();  // the previous iteration's Z is consumed, P1/P2 are loaded
-    // ---- load R token rows as float64 (rows past M are zero)
+    __syncthreads();  // previous Z consumed; factors staged
     for (int ch = tid; ch < R * row_chunks; ch += kThreads) {
-      const int r = ch / row_chunks;
-      double* dst = sm.X + (size_t)ch * 8;
+      const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
+      const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
+      float* dst = X + (size_t)(r * a + i) * L.ldb + q;
       if (r < rows) {
-        load_row_chunk(x + (size_t)m0 * K, ch, dst);
+        load_row_chunk8(x + (size_t)m0 * K, ch, dst);
       } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = 0.0;
+        reinterpret_cast<float4*>(dst)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(dst)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     __syncthreads();
-    // ---- stage 1: Y[(r,i), j] = sum_q X[(r,i), q] P2[q, j]
-    for (int tile = tid; tile < n_tiles; tile += kThreads) {
-      const int rt = tile / ct_n, ct = tile - rt * ct_n;
-      const double* xr = sm.X + (size_t)(rt * 4) * b;
-      double acc[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-      for (int q = 0; q < b; ++q) {
-        double xv[4], pv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) xv[i] = xr[i * b + q];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) pv[j] = sm.P2[q * b + ct + j * ct_n];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fma(xv[i], pv[j], acc[i][j]);
-      }
-      double* yr = sm.Y + (size_t)(rt * 4) * b;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) yr[i * b + ct + j * ct_n] = acc[i][j];
+    // ---- stage 1: Y[(r,i), j] = sum_q X[(r,i), q] P2[q, j]  -> YT[r][j][i]
+    for (int task = warp; task < s1_tasks; task += kWarps) {
+      const int rt = (int)fd_s1ctq.div((uint32_t)task), cq = task - rt * s1_ctq;
+      warp_mma_task<kRotTM, kRotTN>(X, L.ldb, P2T, L.ldb, b, rt * 8 * kRotTM, cq * kRotTN, ct,
+                                    [&](int ri, int j, double v0, double v1) {
+                                      const int r = (int)fd_a.div((uint32_t)ri), i = ri - r * a;
+                                      double* yt = YT + ((size_t)r * b + j) * L.lda + i;
+                                      yt[0] = v0;
+                                      yt[L.lda] = v1;
+                                    });
     }
     __syncthreads();
-    // ---- stage 2: Z[r, i, j] = sum_p P1[p, i] Y[r, p, j], rounded once to float32
-    for (int tile = tid; tile < n_tiles; tile += kThreads) {
-      const int rt = tile / ct_n, ct = tile - rt * ct_n;
-      const int ri0 = rt * 4;
-      const int r = ri0 / a, i0 = ri0 - r * a;
-      const double* yr = sm.Y + (size_t)r * K;
-      double acc[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-      for (int p = 0; p < a; ++p) {
-        double wv[4], yv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) wv[i] = sm.P1[p * a + i0 + i];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) yv[j] = yr[p * b + ct + j * ct_n];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fma(wv[i], yv[j], acc[i][j]);
-      }
-      float* zr = Z + (size_t)ri0 * b;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) zr[i * b + ct + j * ct_n] = __double2float_rn(acc[i][j]);
+    // ---- stage 2: Z[r][i][j] = sum_p P1[p, i] Y[r][p][j], rounded once to float32
+    for (int task = warp; task < s2_tasks; task += kWarps) {
+      const int r = (int)fd_s2tok.div((uint32_t)task);
+      const int rem = task - r * (s2_rt * s1_ctq);
+      const int rt = (int)fd_s1ctq.div((uint32_t)rem), cq = rem - rt * s1_ctq;
+      warp_mma_task<kRotTM, kRotTN>(P1T, L.lda, YT + (size_t)r * b * L.lda, L.lda, a,
+                                    rt * 8 * kRotTM, cq * kRotTN, ct,
+                                    [&](int i, int j, double v0, double v1) {
+                                      float2* z = reinterpret_cast<float2*>(
+                                          Z + (size_t)(r * a + i) * L.ldz + j);
+                                      *z = make_float2(__double2float_rn(v0),
+                                                       __double2float_rn(v1));
+                                    });
     }
     __syncthreads();
-    // ---- epilogue
-    const int n_chunks = R * row_chunks;
+    // ---- epilogue: chunk ch covers elements 8*ch .. 8*ch+7 of the R-row tile
     if (kStoreF32) {
       for (int ch = tid; ch < rows * row_chunks; ch += kThreads) {
-        const float4* src = reinterpret_cast<const float4*>(Z + (size_t)ch * 8);
+        const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
+        const int i = (int)fd_b.div((uint32_t)k8), j = k8 - i * b;
+        const float4* src = reinterpret_cast<const float4*>(Z + (size_t)(r * a + i) * L.ldz + j);
         float4* dst = reinterpret_cast<float4*>(out_f32 + (size_t)m0 * K + (size_t)ch * 8);
         dst[0] = src[0];
         dst[1] = src[1];
       }
     } else {
+      const int n_chunks = R * row_chunks;
       for (int base = 0; base < n_chunks; base += kThreads) {
         const int ch = base + tid;
-        const bool valid = ch < n_chunks && (ch / row_chunks) < rows;
+        const int r = (int)fd_rowc.div((uint32_t)ch);
+        const bool valid = ch < n_chunks && r < rows;
         float v[8];
         if (valid) {
-          const float4* src = reinterpret_cast<const float4*>(Z + (size_t)ch * 8);
-          float4 u0 = src[0], u1 = src[1];
+          const int k8 = (ch - r * row_chunks) * 8;
+          const int i = (int)fd_b.div((uint32_t)k8), j = k8 - i * b;
+          const float4* src =
+              reinterpret_cast<const float4*>(Z + (size_t)(r * a + i) * L.ldz + j);
+          const float4 u0 = src[0], u1 = src[1];
           v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
           v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = 0.f;
+          for (int e = 0; e < 8; ++e) v[e] = 0.f;
         }
         int q[8];
         const float s = quant_group8(v, c, qmax, q);
@@ -326,16 +402,14 @@ int num_sms() {
 }
 
 size_t rotate_smem_bytes(int a, int b, int* rows_per_block) {
-  const size_t fixed = 8u * (size_t)(a * a + b * b);
-  const size_t per_row = 16u * (size_t)(a * b);
-  // prefer two resident blocks per SM (<= 110 KB each), else one (<= 224 KB)
+  // prefer two resident blocks per SM (<= 113 KB each), else one (<= 227 KB)
   int best = 0;
   for (int R = 16; R >= 1; R >>= 1) {
-    if (fixed + per_row * R <= 110u * 1024u) { best = R; break; }
+    if (rot_layout(a, b, R).bytes <= 113u * 1024u) { best = R; break; }
   }
-  if (best == 0 && fixed + per_row <= 224u * 1024u) best = 1;
+  if (best == 0 && rot_layout(a, b, 1).bytes <= 227u * 1024u) best = 1;
   if (rows_per_block) *rows_per_block = best;
-  return best ? fixed + per_row * best : 0;
+  return best ? rot_layout(a, b, best).bytes : 0;
 }
 
 cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, const float* P1,
@@ -358,7 +432,7 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
   int R = 0;
   const size_t smem = rotate_smem_bytes(a, b, &R);
   if (smem == 0) return cudaErrorInvalidValue;
-  const int per_sm = smem <= 110u * 1024u ? 2 : 1;
+  const int per_sm = smem <= 113u * 1024u ? 2 : 1;
   const int64_t want = (M + R - 1) / R;
   const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
   cudaError_t e;
@@ -382,7 +456,7 @@ cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const floa
   int R = 0;
   const size_t smem = rotate_smem_bytes(a, b, &R);
   if (smem == 0) return cudaErrorInvalidValue;
-  const int per_sm = smem <= 110u * 1024u ? 2 : 1;
+  const int per_sm = smem <= 113u * 1024u ? 2 : 1;
   const int grid = (int)std::min<int64_t>((M + R - 1) / R, (int64_t)num_sms() * per_sm);
   auto* k = k_rotate_quant<float, true>;
   cudaError_t e = set_smem(k, smem);

@@ -83,7 +83,7 @@ int64_t lq_act_scale_bytes(int64_t M, int64_t K);
  * Steps 1-3 above for every row of d_x.
  *   d_x      M x K, element type x_dtype (LQ_F32 or LQ_BF16), 16-byte aligned.
  *   d_P1     a x a float32 (row-major) and d_P2 b x b float32, with a*b == K,
- *            a and b multiples of 4 and at most 128.  Pass d_P1 = d_P2 = NULL,
+ *            a a multiple of 16, b of 8, both <= 128.  Pass d_P1 = d_P2 = NULL,
  *            a = b = 0 to skip the rotation (d_x is then the transformed
  *            input x~ itself).  The rotation accumulates in float64 and rounds
  *            once to float32.

@@ -68,7 +68,7 @@ def test_quantize_rejects_bad_arguments_before_launch(L):
     # only one factor
     assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 64, fake, 8, None, 0, 1.0, 4, 32, fake, None,
                              fake, None) == lq.LQ_ERR_ARG
-    # factor sizes not multiples of 4
+    # factor sizes not multiples of 16 (a) and 8 (b)
     assert L.lq_quantize_act(fake, lq.LQ_F32, 4, 96, fake, 6, fake, 16, 1.0, 4, 32, fake, None,
                              fake, None) == lq.LQ_ERR_UNSUPPORTED
     # packed output with 8-bit codes
@@ -95,7 +95,7 @@ def test_weight_entry_points_reject_bad_arguments(L):
     assert L.lq_quantize_weights(fake, 16, 64, 8, 32, fake, None, fake, None) == \
         lq.LQ_ERR_UNSUPPORTED
     # aliasing input and output
-    assert L.lq_fold_weights(fake, 16, 64, fake, 8, fake, 8, fake, None) == lq.LQ_ERR_ARG
+    assert L.lq_fold_weights(fake, 16, 128, fake, 16, fake, 8, fake, None) == lq.LQ_ERR_ARG
     assert L.lq_fold_weights(fake, 16, 64, fake, 4, fake, 8, fake + 16, None) == lq.LQ_ERR_SHAPE
     las = (ctypes.c_float * 2)(1.0, 0.5)
     assert L.lq_layer_create(None, fake, 4, fake, 4, las, 2, 4, ctypes.byref(h)) == lq.LQ_ERR_ARG

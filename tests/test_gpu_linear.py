@@ -42,7 +42,7 @@ def _integer_problem(M, N, K, a_bits, seed):
 def test_gemm_exact_on_integer_problems(a_bits, MNK):
     """With unit steps the library must return the exact integer product."""
     M, N, K = MNK
-    a = 4 if K <= 512 else K // 128
+    a = 16
     b = K // a
     x, w = _integer_problem(M, N, K, a_bits, seed=M + N + K)
     wq = lq.lq_pack_weights(dev(w))
