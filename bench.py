@@ -51,6 +51,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-probe", action="store_true")
+    p.add_argument("--no-aux", action="store_true",
+                   help="skip the quantize-only and decode-GEMV bandwidth measurements")
     return p.parse_args()
 
 
@@ -185,6 +187,18 @@ def cpu_oracle_rate(wl, target_s):
                 tokens_per_s=rows / dt)
 
 
+def max_over_ranks(value_ms, world, device):
+    """Max of a per-rank duration over all ranks (every rank takes part)."""
+    if world <= 1:
+        return float(value_ms)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
@@ -217,6 +231,80 @@ def run_reference(args, rank):
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# HBM-bound kernels of the path, measured on inputs far larger than L2
+# ---------------------------------------------------------------------------
+def aux_hbm_kernels(lq, torch, dev, stream, timed, peaks):
+    out = {}
+    # quantize-only (already transformed fp32 input): 65536 x 2048 fp32 = 512 MiB read
+    M, K = 65536, 2048
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    xt = torch.randn((M, K), generator=g, device=dev, dtype=torch.float32)
+    codes = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sc = torch.empty((M, K // 32), dtype=torch.float32, device=dev)
+
+    def q_step():
+        lq.lq_quantize_act(xt, None, None, 0.85, 4, codes8=codes, scales=sc, stream=stream)
+
+    for _ in range(3):
+        q_step()
+    n = 20
+    ms = timed(n, q_step, flush_between=False) / n
+    byts = M * K * 4 + M * K + M * (K // 32) * 4
+    out["quantize_only"] = {"workload": f"{M}x{K} fp32 -> int8 codes + fp32 steps",
+                            "us": ms * 1e3, "GB_s": byts / (ms * 1e-3) / 1e9,
+                            "frac_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                            "bytes_per_launch": byts}
+    del xt, codes, sc
+    # decode GEMV: W4A8, M = 4 tokens, K = 2048, N = 5632, T = 4 loops over a
+    # stack of 72 distinct resident linears (7.2 MB of packed weights + steps
+    # each, 519 MB in all, > 4x L2), one weight stream per loop and linear
+    wl = synth.decode_workload(4, 5632, 8)
+    (mp,) = synth.module_params(wl)
+    Q1 = lq.lq_inverse_transpose(mp.P1).to(dev)
+    Q2 = lq.lq_inverse_transpose(mp.P2).to(dev)
+    Wf = lq.lq_fold_weights(torch.from_numpy(mp.W).to(dev), Q1, Q2)
+    P1, P2 = torch.from_numpy(mp.P1).to(dev), torch.from_numpy(mp.P2).to(dev)
+    L = 72
+    wqs = [lq.lq_pack_weights(Wf) for _ in range(L)]
+    layers = [lq.lq_layer_create(w, P1, P2, mp.las, 8) for w in wqs]
+    del Wf
+    Md, T = wl.M, wl.T
+    x = torch.from_numpy(np.concatenate([synth.loop_input(wl, wl.linears[0], t).ravel()
+                                         for t in range(T) for _ in range(L)]))
+    x = x.to(torch.bfloat16).to(dev)
+    y = torch.empty(T * L * Md * 5632, dtype=torch.float32, device=dev)
+    ws = lq.workspace(layers, Md, dev)
+
+    def d_step():
+        lq.lq_loop_stack(x, layers, T, lq.LQ_OPEN, M=Md, y=y, ws=ws, stream=stream)
+
+    for _ in range(3):
+        d_step()
+    n = 10
+    step_ms = timed(n, d_step, flush_between=False) / n
+    lq.lq_probe_enable(True)
+    timed(n, d_step, flush_between=False)
+    pr = lq.lq_probe_read()
+    lq.lq_probe_enable(False)
+    gemv_ms, gemv_n = pr["gemv"]
+    per_launch = 5632 * 2048 // 2 + 5632 * 64 * 4 + Md * 2048 + Md * 64 * 4 + Md * 5632 * 4
+    avg = gemv_ms / max(gemv_n, 1)
+    out["gemv_decode"] = {
+        "workload": f"W4A8 M={Md} K=2048 N=5632, T={T} x {L} distinct linears",
+        "gemv_us": avg * 1e3, "GB_s": per_launch / (avg * 1e-3) / 1e9,
+        "frac_hbm": per_launch / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "bytes_per_launch": per_launch,
+        "step_ms": step_ms, "tokens_per_s": Md / (step_ms * 1e-3),
+        "rotate_quantize_us": pr["rotate_quantize"][0] / max(pr["rotate_quantize"][1], 1) * 1e3}
+    for l in layers:
+        l.free()
+    for w in wqs:
+        w.free()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -293,10 +381,7 @@ def run_lq(args, rank, world, local_rank):
     total_ms = timed(args.steps, step)
     clocks = sampler.stop()
     lq.lq_check_device(stream)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
 
     ops_step, rot_step = work_per_step(wl)
     value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
@@ -354,14 +439,14 @@ def run_lq(args, rank, world, local_rank):
             step()
             y_host.copy_(y, non_blocking=True)
 
-        e2e_ms = timed(n_e2e, e2e_step)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(timed(n_e2e, e2e_step), world, dev)
         e2e = {"value": ops_step * n_e2e * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
+
+    aux = None
+    if not args.no_aux:
+        aux = aux_hbm_kernels(lq, torch, dev, stream, timed, load_peaks())
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -382,7 +467,8 @@ def run_lq(args, rank, world, local_rank):
                        "linears": [[lin.name, lin.K, lin.N, lin.a, lin.b] for lin in wl.linears],
                        "x_dtype": wl.x_dtype, "parallelism": f"replicas x{world}",
                        "l2": "flushed between timed steps (256 MiB write outside the events)"},
-            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "kernels": kernels, "aux": aux, "cpu_baseline": cpu,
+            "e2e": e2e,
             "clocks": clocks, "gpu_launches": 2 * T * L * args.steps,
         }
         print(json.dumps(line), flush=True)

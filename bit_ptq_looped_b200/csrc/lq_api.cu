@@ -123,7 +123,7 @@ lq_status check_mk(int64_t M, int64_t K) {
 
 // decode-sized M runs the weight-streaming GEMV while its activation fits in shared memory
 bool use_gemv(int64_t M, int64_t K) {
-  return M <= kGemvMaxM && (size_t)M * (K / kGroup) * 40 <= 200u * 1024u;
+  return M <= kGemvMaxM && K <= 8192 && (size_t)M * (K / kGroup) * 40 <= 200u * 1024u;
 }
 
 int64_t ws_bytes_for(int64_t M, int64_t K) {
@@ -752,6 +752,16 @@ lq_status lq_probe_read(double* h_ms, int64_t* h_count) {
     g_probe.pending[k].clear();
   }
   return st;
+}
+
+lq_status lq_selftest_bounded_wait(int64_t limit_us, void* stream) {
+  if (limit_us <= 0 || limit_us > 10000000) {
+    set_error("limit must be in (0, 10 s]");
+    return LQ_ERR_ARG;
+  }
+  cudaError_t e = launch_wait_selftest((uint64_t)limit_us * 1000u, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_error(e, "self-test launch");
+  return LQ_OK;
 }
 
 lq_status lq_check_device(void* stream) {

@@ -264,6 +264,7 @@ cudaError_t launch_group_gemm(const uint8_t* A, const float* sa, const uint8_t* 
                               const float* sw_t, float* y, int64_t M, int64_t N, int64_t K,
                               int opf, cudaStream_t s, const char** why);
 lq_status read_and_clear_device_status(cudaStream_t s);
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
 
 // GEMV (lq_gemv.cu)
 cudaError_t launch_group_gemv(const int8_t* qa, const float* sa, const uint8_t* w4,

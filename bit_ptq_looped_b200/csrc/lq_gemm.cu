@@ -362,6 +362,26 @@ cudaError_t launch_group_gemm(const uint8_t* A, const float* sa, const uint8_t* 
   return launch_impl<1>(A, sa, B, sw_t, y, M, N, K, s, why);
 }
 
+namespace {
+// One thread waits on an mbarrier phase that nothing completes, through the
+// same bounded wait the GEMM roles use; it gives up after limit_ns.
+__global__ void k_wait_selftest(uint64_t limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  mbar_wait_bounded(b, 0u, &abort_flag, &g_gemm_status, limit_ns);
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s) {
+  k_wait_selftest<<<1, 32, 0, s>>>(limit_ns);
+  return cudaGetLastError();
+}
+
 lq_status read_and_clear_device_status(cudaStream_t s) {
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_error(e, "stream synchronize");
@@ -371,7 +391,7 @@ lq_status read_and_clear_device_status(cudaStream_t s) {
   if (v != 0) {
     e = cudaMemcpyToSymbol(g_gemm_status, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_error(e, "clear device status");
-    set_error("a bounded device-side wait expired (status %d)", v);
+    set_error("a bounded device-side wait expired in the GEMM kernel (status %d)", v);
     return (lq_status)v;
   }
   return LQ_OK;

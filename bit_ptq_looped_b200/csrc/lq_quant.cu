@@ -50,15 +50,19 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* __restrict__ x, int64
 // Quantize the 8 values a thread holds; the 4 consecutive lanes 4j..4j+3 of
 // a warp hold one group of 32.  Every lane of the warp must call this.
 //
-// The code is rne(fl32(x / s)), decided without a division per element:
-// r1 = fl32(x * fl32(1 / s)) lies within 1.5 ulp of fl32(x / s), so the two
-// round to the same integer unless a half-integer lies within that distance
-// of r1.  Values within 2^-14 of a half-integer (far more than 1.5 ulp for
-// every |r1| < 128, the range that can round inside [-q_max, q_max]) take the
-// true IEEE division instead; NaN or infinite r1 (s so small that 1 / s
-// overflows) fails the same test and takes it too.
+// The code is rne(fl32(x / s)) clamped to [-q_max, q_max], decided without a
+// division per element: r1 = fl32(x * fl32(1 / s)) lies within 1.5 ulp of
+// fl32(x / s), so the two round to the same integer unless a half-integer
+// lies within that distance of r1.  Values within 2^-14 of a half-integer
+// (far more than 1.5 ulp for |r1| < 128, the range that can round inside
+// [-q_max, q_max]) take the true IEEE division instead, and so does a whole
+// group whose 1 / s overflows.  Clamping before rounding gives the same code
+// (the bounds are integers).  Adding 1.5 * 2^23 rounds to the nearest integer
+// (ties to even) and leaves the code's two's-complement byte in the low bits.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
 __device__ __forceinline__ float quant_group8(const float (&v)[8], float c, int qmax,
-                                              int (&q)[8]) {
+                                              uint32_t (&qb)[8]) {
   float am = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
@@ -67,21 +71,61 @@ __device__ __forceinline__ float quant_group8(const float (&v)[8], float c, int 
   // s = fl32(fl32(c * absmax) / q_max): two IEEE round-to-nearest operations
   const float s = __fdiv_rn(__fmul_rn(c, am), (float)qmax);
   const float inv = __frcp_rn(s);
+  const float qm = (float)qmax;
+  const bool slow_group = !(inv <= 3.0e38f);  // 1/s overflowed (or s == 0)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    int qi = 0;
-    if (s != 0.f) {
-      const float r1 = __fmul_rn(v[i], inv);
-      const float rr = rintf(r1);
-      const float tie_dist = 0.5f - fabsf(r1 - rr);
-      float r = rr;
-      if (!(tie_dist > 6.103515625e-05f))  // 2^-14, or NaN
-        r = rintf(__fdiv_rn(v[i], s));     // fl32(x / s), true division, then RNE
-      qi = (int)fminf(fmaxf(r, (float)-qmax), (float)qmax);
+    const float r1 = fminf(fmaxf(__fmul_rn(v[i], inv), -qm), qm);
+    float f = __fadd_rn(r1, kRoundMagic);
+    const float rr = __fsub_rn(f, kRoundMagic);
+    const float tie_dist = 0.5f - fabsf(r1 - rr);
+    if (slow_group || !(tie_dist > 6.103515625e-05f)) {  // 2^-14
+      const float r = s != 0.f ? fminf(fmaxf(__fdiv_rn(v[i], s), -qm), qm) : 0.f;
+      f = __fadd_rn(r, kRoundMagic);  // fl32(x / s), then RNE
     }
-    q[i] = qi;
+    qb[i] = __float_as_uint(f);
   }
   return s;
+}
+
+// two's-complement code bytes (low byte of each qb) -> one 32-bit word
+__device__ __forceinline__ uint32_t pack_bytes4(uint32_t b0, uint32_t b1, uint32_t b2,
+                                                uint32_t b3) {
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// E4M3 byte of an integer code |q| <= 7 held as the low byte of qb
+__device__ __forceinline__ uint32_t e4m3_byte(uint32_t qb) {
+  const int q = (int)(int8_t)(qb & 0xFFu);
+  const uint32_t mag = (uint32_t)(q < 0 ? -q : q);
+  const uint32_t byte = __byte_perm((uint32_t)(kE4M3Int0to7 & 0xFFFFFFFFull),
+                                    (uint32_t)(kE4M3Int0to7 >> 32), mag) & 0xFFu;
+  return byte | (q < 0 ? 0x80u : 0u);
+}
+
+// Write one thread's 8 codes (and its group's step from lane 4j).
+__device__ __forceinline__ void store_codes(const uint32_t (&qb)[8], float s, int64_t chunk,
+                                            int8_t* __restrict__ codes8, int opf,
+                                            uint8_t* __restrict__ codes4,
+                                            float* __restrict__ scales) {
+  if (codes8) {
+    uint2 w;
+    if (opf == kOpE4M3) {
+      w.x = pack_bytes4(e4m3_byte(qb[0]), e4m3_byte(qb[1]), e4m3_byte(qb[2]), e4m3_byte(qb[3]));
+      w.y = pack_bytes4(e4m3_byte(qb[4]), e4m3_byte(qb[5]), e4m3_byte(qb[6]), e4m3_byte(qb[7]));
+    } else {
+      w.x = pack_bytes4(qb[0], qb[1], qb[2], qb[3]);
+      w.y = pack_bytes4(qb[4], qb[5], qb[6], qb[7]);
+    }
+    reinterpret_cast<uint2*>(codes8)[chunk] = w;
+  }
+  if (codes4) {
+    uint32_t p = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) p |= (qb[j] & 0xFu) << (4 * j);
+    reinterpret_cast<uint32_t*>(codes4)[chunk] = p;
+  }
+  if ((threadIdx.x & 3) == 0) scales[chunk >> 2] = s;
 }
 
 // floor(n / d) for n, d < 2^16 with one multiply-high (d fixed per launch)
@@ -91,54 +135,35 @@ struct FastDiv {
   __device__ __forceinline__ uint32_t div(uint32_t n) const { return d == 1u ? n : __umulhi(n, m); }
 };
 
-// Write one thread's 8 codes (and its group's step from lane 4j).
-__device__ __forceinline__ void store_codes(const int (&q)[8], float s, int64_t chunk,
-                                            int8_t* __restrict__ codes8, int opf,
-                                            uint8_t* __restrict__ codes4,
-                                            float* __restrict__ scales) {
-  if (codes8) {
-    uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      w0 |= encode_code_byte(q[i], opf) << (8 * i);
-      w1 |= encode_code_byte(q[i + 4], opf) << (8 * i);
-    }
-    reinterpret_cast<uint2*>(codes8)[chunk] = make_uint2(w0, w1);
-  }
-  if (codes4) {
-    uint32_t p = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = (uint32_t)q[2 * j] & 0xFu, hi = (uint32_t)q[2 * j + 1] & 0xFu;
-      p |= (lo | (hi << 4)) << (8 * j);
-    }
-    reinterpret_cast<uint32_t*>(codes4)[chunk] = p;
-  }
-  if ((threadIdx.x & 3) == 0) scales[chunk >> 2] = s;
-}
-
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) k_quant_only(const Tin* __restrict__ x,
                                                          int64_t n_chunks, float c, int qmax,
                                                          int8_t* __restrict__ codes8, int opf,
                                                          uint8_t* __restrict__ codes4,
                                                          float* __restrict__ scales) {
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  // n_chunks is a multiple of 4 and the loop bound is warp-uniform, so the
-  // 4 lanes of a group are all valid or all invalid
-  for (int64_t base = (int64_t)blockIdx.x * kThreads; base < n_chunks; base += stride) {
-    const int64_t ch = base + threadIdx.x;
-    const bool valid = ch < n_chunks;
-    float v[8];
-    if (valid) {
-      load8(x, ch, v);
-    } else {
+  // Two 8-element chunks per thread per step (blockDim apart) keep more loads
+  // in flight.  n_chunks is a multiple of 4 and every bound below is
+  // warp-uniform, so the 4 lanes of a group are all valid or all invalid.
+  const int64_t stride = (int64_t)gridDim.x * (2 * kThreads);
+  for (int64_t base = (int64_t)blockIdx.x * (2 * kThreads); base < n_chunks; base += stride) {
+    const int64_t ch0 = base + threadIdx.x, ch1 = ch0 + kThreads;
+    const bool v0 = ch0 < n_chunks, v1 = ch1 < n_chunks;
+    float a0[8], a1[8];
+    if (v0) load8(x, ch0, a0);
+    if (v1) load8(x, ch1, a1);
+    if (!v0) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      for (int i = 0; i < 8; ++i) a0[i] = 0.f;
     }
-    int q[8];
-    const float s = quant_group8(v, c, qmax, q);
-    if (valid) store_codes(q, s, ch, codes8, opf, codes4, scales);
+    if (!v1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a1[i] = 0.f;
+    }
+    uint32_t q0[8], q1[8];
+    const float s0 = quant_group8(a0, c, qmax, q0);
+    const float s1 = quant_group8(a1, c, qmax, q1);
+    if (v0) store_codes(q0, s0, ch0, codes8, opf, codes4, scales);
+    if (v1) store_codes(q1, s1, ch1, codes8, opf, codes4, scales);
   }
 }
 
@@ -342,7 +367,7 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = 0.f;
         }
-        int q[8];
+        uint32_t q[8];
         const float s = quant_group8(v, c, qmax, q);
         if (valid) store_codes(q, s, m0 * row_chunks + ch, codes8, opf, codes4, scales);
       }
@@ -419,7 +444,7 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
   if (M == 0) return cudaSuccess;
   if (P1 == nullptr) {
     const int64_t n_chunks = M * K / 8;
-    const int64_t want = (n_chunks + kThreads - 1) / kThreads;
+    const int64_t want = (n_chunks + 2 * kThreads - 1) / (2 * kThreads);
     const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * 8);
     if (x_dtype == LQ_BF16)
       k_quant_only<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
@@ -430,8 +455,12 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
     return cudaGetLastError();
   }
   int R = 0;
-  const size_t smem = rotate_smem_bytes(a, b, &R);
+  size_t smem = rotate_smem_bytes(a, b, &R);
   if (smem == 0) return cudaErrorInvalidValue;
+  if (M < (int64_t)R * num_sms()) {  // too few rows to fill the GPU: one row per block
+    R = 1;
+    smem = rot_layout(a, b, 1).bytes;
+  }
   const int per_sm = smem <= 113u * 1024u ? 2 : 1;
   const int64_t want = (M + R - 1) / R;
   const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
@@ -454,8 +483,12 @@ cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const floa
                                 const float* Q2, int b, float* out, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   int R = 0;
-  const size_t smem = rotate_smem_bytes(a, b, &R);
+  size_t smem = rotate_smem_bytes(a, b, &R);
   if (smem == 0) return cudaErrorInvalidValue;
+  if (M < (int64_t)R * num_sms()) {  // too few rows to fill the GPU: one row per block
+    R = 1;
+    smem = rot_layout(a, b, 1).bytes;
+  }
   const int per_sm = smem <= 113u * 1024u ? 2 : 1;
   const int grid = (int)std::min<int64_t>((M + R - 1) / R, (int64_t)num_sms() * per_sm);
   auto* k = k_rotate_quant<float, true>;

@@ -48,6 +48,7 @@ SIGNATURES = {
     "lq_loop_linear": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
     "lq_check_device": (_i32, [_vp]),
+    "lq_selftest_bounded_wait": (_i32, [_i64, _vp]),
     "lq_loop_linear_noalloc": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp]),
     "lq_probe_enable": (_i32, [_i32]),
     "lq_probe_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]),
@@ -331,3 +332,7 @@ def lq_probe_read() -> dict:
     cnt = (_i64 * len(PROBE_KINDS))()
     _check(lib().lq_probe_read(ms, cnt), "lq_probe_read")
     return {k: (ms[i], cnt[i]) for i, k in enumerate(PROBE_KINDS)}
+
+
+def lq_selftest_bounded_wait(limit_us: int = 1000, stream=None) -> None:
+    _check(lib().lq_selftest_bounded_wait(limit_us, _stream(stream)), "lq_selftest_bounded_wait")

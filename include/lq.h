@@ -242,6 +242,16 @@ lq_status lq_probe_read(double* h_ms, int64_t* h_count);
  */
 lq_status lq_check_device(void* stream);
 
+/*
+ * lq_selftest_bounded_wait -- diagnostic of the failure path: enqueue a tiny
+ * kernel that waits, through the same bounded mbarrier wait the GEMM uses, on
+ * a barrier phase that nothing completes.  The wait gives up after limit_us
+ * microseconds (0 < limit_us <= 10 s) and records LQ_ERR_DEVICE_TIMEOUT in the
+ * device status word; the kernel then returns normally and the context stays
+ * usable.  A following lq_check_device(stream) reports (and clears) it.
+ */
+lq_status lq_selftest_bounded_wait(int64_t limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
