@@ -21,8 +21,9 @@
 //
 // Warp roles (576 threads): warps 0-15 epilogue, warp 16 TMA producer, warp
 // 17 MMA issuer.  Epilogue warp w reads TMEM lane quadrant w % 4 (its 32 rows)
-// and the 32-column block w / 4 of every group's accumulator with one load,
-// releases the buffer, and folds the columns with packed f32x2 arithmetic.
+// and the 32-column block w / 4 of the accumulators, two groups at a time (one
+// barrier wait per pair), releases the buffers, and folds the columns with
+// packed f32x2 arithmetic.
 // (Variants that pipelined the TMEM loads across pieces or groups, split the
 // groups between two warp sets, or ran two CTAs per SM measured no faster.)
 // Every mbarrier wait is bounded; on expiry the kernel records
@@ -225,7 +226,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------- epilogue: warps 0..EPI_WARPS-1 ----------------
-    static_assert(EPI_COLS == 32, "one 32-column TMEM load per group");
+    // Groups are folded in pairs (gi, gi + 1) of the same stage.  The MMAs of a
+    // CTA retire in issue order, so the barrier of group gi + 1 covers both.
+    static_assert(EPI_COLS == 32 && GPS % 2 == 0, "pairs of groups, two 16-column halves");
     const int quad = warp & 3;
     const int col0 = (warp >> 2) * EPI_COLS;
     const int row = quad * 32 + lane;
@@ -234,36 +237,52 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int i = 0; i < EPI_COLS / 2; ++i) acc[i] = make_float2(0.f, 0.f);
     bool ok = true;
-    for (int gi = 0; gi < G && ok; ++gi) {
+    for (int gi = 0; gi < G && ok; gi += 2) {
       const int kb = gi / GPS, j = gi % GPS, st = kb % STAGES;
-      if (j == 0)  // the group's steps arrive with its stage
+      if (j == 0)  // the pair's steps arrive with its stage
         ok = mbar_wait_bounded(bar_full + 8 * st, (uint32_t)(kb / STAGES) & 1u, abort_flag,
                                &g_gemm_status, kWaitLimitNs);
-      const int buf = gi % ACC_BUFS;
-      ok = ok && mbar_wait_bounded(bar_accf + 8 * buf, (uint32_t)(gi / ACC_BUFS) & 1u,
+      const int b0 = gi % ACC_BUFS, b1 = (gi + 1) % ACC_BUFS;
+      ok = ok && mbar_wait_bounded(bar_accf + 8 * b1, (uint32_t)((gi + 1) / ACC_BUFS) & 1u,
                                    abort_flag, &g_gemm_status, kWaitLimitNs);
       if (!ok) break;
       tc_fence_after();
-      uint32_t r[EPI_COLS];
-      tmem_ld_32x32b_x32(lane_base + (uint32_t)(buf * BN), r);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acce + 8 * buf);  // accumulator buffer is free again
-      const float s_a =
-          reinterpret_cast<const float*>(gbase + OFF_SA + st * SA_BYTES + row * 16)[j];
-      const float2 s2 = make_float2(s_a, s_a);
-      const float4* swv =
+      const float* sa_row = reinterpret_cast<const float*>(gbase + OFF_SA + st * SA_BYTES) + row * 4;
+      const float sa0 = sa_row[j], sa1 = sa_row[j + 1];
+      const float2 s20 = make_float2(sa0, sa0), s21 = make_float2(sa1, sa1);
+      const float4* sw0 =
           reinterpret_cast<const float4*>(gbase + OFF_SW + st * SW_BYTES) + (j * BN + col0) / 4;
+      const float4* sw1 = sw0 + BN / 4;
+      uint32_t rA[16], rB[16];
 #pragma unroll
-      for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
-        const float4 w = swv[c4];
-        acc[2 * c4] = ffma2(fmul2(s2, make_float2(w.x, w.y)),
-                            acc_pair<kKindI8>(r[4 * c4 + 0], r[4 * c4 + 1]), acc[2 * c4]);
-        acc[2 * c4 + 1] = ffma2(fmul2(s2, make_float2(w.z, w.w)),
-                                acc_pair<kKindI8>(r[4 * c4 + 2], r[4 * c4 + 3]), acc[2 * c4 + 1]);
+      for (int h = 0; h < 2; ++h) {  // column halves 0-15, 16-31
+        tmem_ld_32x32b_x16(lane_base + (uint32_t)(b0 * BN + 16 * h), rA);
+        tmem_ld_32x32b_x16(lane_base + (uint32_t)(b1 * BN + 16 * h), rB);
+        tmem_wait_ld();
+        if (h == 1) {  // both accumulators fully read: hand the buffers back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(bar_acce + 8 * b0);
+            mbar_arrive(bar_acce + 8 * b1);
+          }
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const float4 w0 = sw0[4 * h + c4], w1 = sw1[4 * h + c4];
+          float2& a0 = acc[8 * h + 2 * c4];
+          float2& a1 = acc[8 * h + 2 * c4 + 1];
+          a0 = ffma2(fmul2(s20, make_float2(w0.x, w0.y)),
+                     acc_pair<kKindI8>(rA[4 * c4 + 0], rA[4 * c4 + 1]), a0);
+          a1 = ffma2(fmul2(s20, make_float2(w0.z, w0.w)),
+                     acc_pair<kKindI8>(rA[4 * c4 + 2], rA[4 * c4 + 3]), a1);
+          a0 = ffma2(fmul2(s21, make_float2(w1.x, w1.y)),
+                     acc_pair<kKindI8>(rB[4 * c4 + 0], rB[4 * c4 + 1]), a0);
+          a1 = ffma2(fmul2(s21, make_float2(w1.z, w1.w)),
+                     acc_pair<kKindI8>(rB[4 * c4 + 2], rB[4 * c4 + 3]), a1);
+        }
       }
-      if (j == GPS - 1) {  // this stage's shared-memory steps are no longer needed
+      if (j + 2 == GPS) {  // this stage's shared-memory steps are no longer needed
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty + 8 * st);
       }
