@@ -37,6 +37,7 @@ METRIC = "W4A4 looped-linear TOPS & tokens/s at 1 B200; % of int8 tensor/HBM roo
 SM_COUNT = 148
 SM_CLOCK_GHZ = 1.965
 FP64_FMA_PER_SM_CLK = 64  # B200 FP64 units per SM
+FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM
 
 
 def parse_args():
@@ -291,7 +292,7 @@ def aux_hbm_kernels(lq, torch, dev, stream, timed, peaks):
     pr = lq.lq_probe_read()
     lq.lq_probe_enable(False)
     gemv_ms, gemv_n = pr["gemv"]
-    per_launch = 5632 * 2048 // 2 + 5632 * 64 * 4 + Md * 2048 + Md * 64 * 4 + Md * 5632 * 4
+    per_launch = 5632 * 2048 // 2 + 5632 * 64 * 4 + Md * 2048 + Md * 64 * 8 + Md * 5632 * 4
     avg = gemv_ms / max(gemv_n, 1)
     out["gemv_decode"] = {
         "workload": f"W4A8 M={Md} K=2048 N=5632, T={T} x {L} distinct linears",
@@ -299,6 +300,9 @@ def aux_hbm_kernels(lq, torch, dev, stream, timed, peaks):
         "frac_hbm": per_launch / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "bytes_per_launch": per_launch,
         "step_ms": step_ms, "tokens_per_s": Md / (step_ms * 1e-3),
+        # the whole stack as one weight stream: T x L launches' bytes over the step
+        "stream_GB_s": T * L * per_launch / (step_ms * 1e-3) / 1e9,
+        "stream_frac_hbm": T * L * per_launch / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "rotate_quantize_us": pr["rotate_quantize"][0] / max(pr["rotate_quantize"][1], 1) * 1e3}
     for l in layers:
         l.free()
@@ -345,7 +349,9 @@ def run_lq(args, rank, world, local_rank):
     n_out = T * M * sum(lin.N for lin in wl.linears)
     y = torch.empty(n_out, dtype=torch.float32, device=dev)
     y_host = torch.empty(n_out, dtype=torch.float32).pin_memory()
-    ws = lq.workspace(layers, M, dev)
+    # open mode with a workspace for all T loops: one quantize and one GEMM
+    # launch per linear cover the T loops (the loops are independent here)
+    ws = lq.workspace(layers, M, dev, T=T)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
 
@@ -384,6 +390,7 @@ def run_lq(args, rank, world, local_rank):
     total_ms = max_over_ranks(total_ms, world, dev)
 
     ops_step, rot_step = work_per_step(wl)
+    loops_per_launch = min(T, 8) if M > 16 else 1  # the driver's open-mode batching
     value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
     ms_per_step = total_ms / args.steps
     tokens_per_s = M * args.steps * world / (total_ms * 1e-3)
@@ -405,29 +412,36 @@ def run_lq(args, rank, world, local_rank):
         for v in kernels.values():
             v["share"] = v["avg_us"] * v["launches"] / tot
         dom = max(kernels, key=lambda k: kernels[k]["avg_us"] * kernels[k]["launches"])
-        per_launch = {lin.name: lin for lin in wl.linears}
         avg_s = kernels[dom]["avg_us"] * 1e-6
-        n_lin = len(wl.linears)
+        per_step = kernels[dom]["launches"] / n_probe  # launches of that kind per step
         if dom == "gemm":
-            flops = sum(2 * M * lin.N * lin.K for lin in wl.linears) / n_lin
+            flops = sum(2 * M * lin.N * lin.K * T for lin in wl.linears) / per_step
             peak = 2.0 * peaks["bf16_tflops"]  # 8-bit dense = 2x bf16 dense (nominal ratio)
             roofline = {"bound": "tensor", "achieved": flops / avg_s / 1e12, "peak": peak,
                         "unit": "TFLOP/s", "peak_source": peaks["source"] +
                         " bf16 burst x2 (8-bit/16-bit nominal ratio)"}
+            # the unit that binds this kernel: the fp32 group rescale, 2 lane
+            # operations (s_a*s_w, then the fused multiply-add) per output and group
+            epi = sum(2 * M * lin.N * (lin.K // 32) * T for lin in wl.linears) / per_step
+            epi_peak = SM_COUNT * FP32_LANES_PER_SM * SM_CLOCK_GHZ * 1e9 / 1e12
+            roofline["epilogue_alu"] = {
+                "achieved": epi / avg_s / 1e12, "peak": epi_peak, "unit": "T lane-ops/s",
+                "frac": epi / avg_s / 1e12 / epi_peak,
+                "peak_source": "derived: 148 SM x 128 FP32 lanes x 1.965 GHz"}
         elif dom == "rotate_quantize":
-            flops = sum(2 * M * lin.K * (lin.a + lin.b) for lin in wl.linears) / n_lin
+            flops = sum(2 * M * lin.K * (lin.a + lin.b) * T for lin in wl.linears) / per_step
             peak = SM_COUNT * FP64_FMA_PER_SM_CLK * 2 * SM_CLOCK_GHZ * 1e9 / 1e12
             roofline = {"bound": "alu", "achieved": flops / avg_s / 1e12, "peak": peak,
                         "unit": "TFLOP/s", "peak_source":
                         "derived: 148 SM x 64 FP64 FMA/clk x 2 x 1.965 GHz"}
         else:
-            byts = sum(lin.N * lin.K // 2 + lin.N * lin.K // 8 for lin in wl.linears) / n_lin
+            byts = sum((lin.N * lin.K // 2 + lin.N * lin.K // 8) * T
+                       for lin in wl.linears) / per_step
             roofline = {"bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "peak_source": peaks["source"]}
         roofline["frac"] = roofline["achieved"] / roofline["peak"]
         roofline["kernel"] = dom
         roofline["traffic"] = ncu_traffic(dom, wl.name)
-        del per_launch
 
     # end to end through the public API with host buffers
     e2e = None
@@ -466,10 +480,11 @@ def run_lq(args, rank, world, local_rank):
             "config": {"workload": wl.name, "M": M, "T": T, "a_bits": wl.a_bits, "group": 32,
                        "linears": [[lin.name, lin.K, lin.N, lin.a, lin.b] for lin in wl.linears],
                        "x_dtype": wl.x_dtype, "parallelism": f"replicas x{world}",
+                       "loops_per_launch": loops_per_launch,
                        "l2": "flushed between timed steps (256 MiB write outside the events)"},
             "roofline": roofline, "kernels": kernels, "aux": aux, "cpu_baseline": cpu,
             "e2e": e2e,
-            "clocks": clocks, "gpu_launches": 2 * T * L * args.steps,
+            "clocks": clocks, "gpu_launches": 2 * L * -(-T // loops_per_launch) * args.steps,
         }
         print(json.dumps(line), flush=True)
     for l in layers:

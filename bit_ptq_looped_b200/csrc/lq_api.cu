@@ -126,8 +126,11 @@ bool use_gemv(int64_t M, int64_t K) {
   return M <= kGemvMaxM && K <= 8192 && (size_t)M * (K / kGroup) * 40 <= 200u * 1024u;
 }
 
+// workspace: codes (M x K bytes), steps (M x G fp32), and for the GEMV path the
+// per-group code sums (M x G int32)
 int64_t ws_bytes_for(int64_t M, int64_t K) {
-  return round_up(M * K, 256) + round_up(M * (K / kGroup) * 4, 256);
+  const int64_t steps = round_up(M * (K / kGroup) * 4, 256);
+  return round_up(M * K, 256) + steps + (use_gemv(M, K) ? steps : 0);
 }
 
 // Graph cache of the loop driver: one instantiated graph per argument set.
@@ -213,30 +216,58 @@ struct ProbeScope {
   }
 };
 
-// one application of a layer: quantize into the workspace, then GEMM / GEMV
+bool probe_on() {
+  std::lock_guard<std::mutex> lk(g_probe.mu);
+  return g_probe.on;
+}
+
+// Enqueue one looped linear (quantize, then GEMV or GEMM) for loops
+// t .. t + nb - 1 of one layer: launch row r is row r % M of loop t + r / M,
+// whose input starts x_stride elements after the previous loop's and whose
+// output starts y_stride floats after it (nb = 1: one loop, strides unused).
+// pdl_first: the quantizer may overlap the previous kernel of the same
+// sequence (programmatic dependent launch); x_early: x was written before the
+// sequence began.  The consumer kernel always overlaps the quantizer's tail.
 lq_status enqueue_linear(const void* x, int32_t x_dtype, int64_t M, const lq_layer* L, int t,
-                         float* y, void* ws, cudaStream_t s) {
+                         float* y, void* ws, cudaStream_t s, bool pdl_first = false,
+                         bool x_early = true, int nb = 1, int64_t x_stride = 0,
+                         int64_t y_stride = 0) {
   const lq_wq* wq = L->wq;
-  const int64_t K = wq->K, N = wq->N;
-  const bool gemv = use_gemv(M, K);
-  const int opf = gemv ? kOpInt8 : (L->a_bits == 4 ? kOpE4M3 : kOpInt8);
+  const int64_t K = wq->K, N = wq->N, Mt = M * nb;
+  const bool gemv = use_gemv(Mt, K);
+  const int opf = gemv ? kOpGemvAct : (L->a_bits == 4 ? kOpE4M3 : kOpInt8);
   uint8_t* codes = (uint8_t*)ws;
-  float* scales = (float*)((char*)ws + round_up(M * K, 256));
+  float* scales = (float*)((char*)ws + round_up(Mt * K, 256));
+  int* asum = gemv ? (int*)((char*)scales + round_up(Mt * (K / kGroup) * 4, 256)) : nullptr;
+  if (nb > 1 && (gemv || L->P1 == nullptr || nb > kMaxLoopsPerLaunch)) {
+    set_error("internal: loop batching needs the rotating tensor-core path");
+    return LQ_ERR_ARG;
+  }
+  LoopSegs segs = one_loop(L->las[t]);
+  if (nb > 1) {
+    segs.seg_rows = M;
+    segs.x_stride = x_stride;
+    for (int j = 0; j < nb; ++j) segs.c[j] = L->las[t + j];
+  }
+  // no programmatic overlap while the probe brackets each kernel with events
+  const bool pdl = !probe_on();
   cudaError_t e;
   {
     ProbeScope ps(kProbeRotQuant, s);
-    e = launch_quantize(x, x_dtype, M, K, L->P1, L->a, L->P2, L->b, L->las[t], L->a_bits,
-                        (int8_t*)codes, opf, nullptr, scales, s);
+    e = launch_quantize(x, x_dtype, Mt, K, L->P1, L->a, L->P2, L->b, segs, L->a_bits,
+                        (int8_t*)codes, opf, nullptr, scales, s, pdl && pdl_first, x_early, asum);
   }
   if (e != cudaSuccess) return cuda_error(e, "quantize launch");
   if (gemv) {
     ProbeScope ps(kProbeGemv, s);
-    e = launch_group_gemv((const int8_t*)codes, scales, wq->codes4, wq->scales, y, M, N, K, s);
+    e = launch_group_gemv((const int8_t*)codes, asum, scales, wq->codes4, wq->scales, y, M, N, K,
+                          s, pdl);
     if (e != cudaSuccess) return cuda_error(e, "gemv launch");
   } else {
     ProbeScope ps(kProbeGemm, s);
     const char* why = nullptr;
-    e = launch_group_gemm(codes, scales, wq->op[opf], wq->scales_t, y, M, N, K, opf, s, &why);
+    e = launch_group_gemm(codes, scales, wq->op[opf], wq->scales_t, y, Mt, N, K, opf, s, &why,
+                          pdl, nb > 1 ? M : INT64_MAX, y_stride);
     if (e != cudaSuccess) {
       if (why) {
         set_error("gemm launch: %s", why);
@@ -246,6 +277,17 @@ lq_status enqueue_linear(const void* x, int32_t x_dtype, int64_t M, const lq_lay
     }
   }
   return LQ_OK;
+}
+
+// Loops of one layer that open mode runs per launch with a workspace of
+// ws_bytes: batching needs the rotating tensor-core path for M rows.
+int loops_per_launch(const lq_layer* L, int64_t M, int T, int64_t ws_bytes) {
+  const int64_t K = L->wq->K;
+  if (use_gemv(M, K) || L->P1 == nullptr) return 1;
+  int nb = std::min(T, kMaxLoopsPerLaunch);
+  while (nb > 1 && (ws_bytes_for(M * nb, K) > ws_bytes || M * nb > ((int64_t)1 << 31) - 256))
+    --nb;
+  return nb;
 }
 
 lq_status check_layer_call(const lq_layer* layer, int64_t M, int32_t x_dtype) {
@@ -316,8 +358,8 @@ lq_status lq_quantize_act(const void* d_x, int32_t x_dtype, int64_t M, int64_t K
     set_error("input and output pointers must be 16-byte aligned");
     return LQ_ERR_ALIGN;
   }
-  cudaError_t e = launch_quantize(d_x, x_dtype, M, K, d_P1, a, d_P2, b, las_t, bits, d_codes8,
-                                  kOpInt8, d_codes4, d_scales, (cudaStream_t)stream);
+  cudaError_t e = launch_quantize(d_x, x_dtype, M, K, d_P1, a, d_P2, b, one_loop(las_t), bits,
+                                  d_codes8, kOpInt8, d_codes4, d_scales, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_error(e, "quantize launch");
   return LQ_OK;
 }
@@ -408,8 +450,8 @@ lq_status lq_quantize_weights(const float* d_W, int64_t N, int64_t K, int32_t bi
     set_error("pointers must be 16-byte aligned");
     return LQ_ERR_ALIGN;
   }
-  cudaError_t e = launch_quantize(d_W, LQ_F32, N, K, nullptr, 0, nullptr, 0, 1.0f, 4, d_codes8,
-                                  kOpInt8, d_codes4, d_scales, (cudaStream_t)stream);
+  cudaError_t e = launch_quantize(d_W, LQ_F32, N, K, nullptr, 0, nullptr, 0, one_loop(1.0f), 4,
+                                  d_codes8, kOpInt8, d_codes4, d_scales, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_error(e, "weight quantize launch");
   return LQ_OK;
 }
@@ -452,8 +494,8 @@ lq_status lq_pack_weights(const float* d_W_folded, int64_t N, int64_t K, int32_t
     return LQ_ERR_NOMEM;
   }
   w->bytes = (int64_t)(b4 + 2 * bs);
-  e = launch_quantize(d_W_folded, LQ_F32, N, K, nullptr, 0, nullptr, 0, 1.0f, 4, nullptr,
-                      kOpInt8, w->codes4, w->scales, s);
+  e = launch_quantize(d_W_folded, LQ_F32, N, K, nullptr, 0, nullptr, 0, one_loop(1.0f), 4,
+                      nullptr, kOpInt8, w->codes4, w->scales, s);
   if (e == cudaSuccess) e = launch_transpose_f32(w->scales, N, w->G, w->scales_t, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
@@ -573,6 +615,20 @@ int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M) 
   return need;
 }
 
+int64_t lq_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M,
+                                 int32_t T) {
+  if (!layers || L <= 0 || M < 0 || T <= 0) return -1;
+  int64_t need = 0;
+  for (int i = 0; i < L; ++i) {
+    if (!layers[i]) return -1;
+    const int64_t K = layers[i]->wq->K;
+    const bool batch = !use_gemv(M, K) && layers[i]->P1 != nullptr;
+    const int nb = batch ? std::min<int>(T, kMaxLoopsPerLaunch) : 1;
+    need = std::max(need, ws_bytes_for(M * nb, K));
+  }
+  return need;
+}
+
 lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_layer* layer,
                          int32_t t, float* d_y, void* d_ws, int64_t ws_bytes, void* stream) {
   lq_status st;
@@ -600,24 +656,48 @@ lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_l
 
 static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
                                const lq_layer* const* layers, int32_t L, int32_t T, int32_t mode,
-                               float* d_y, void* d_ws, cudaStream_t s) {
-  const char* xcur = (const char*)d_x;
+                               float* d_y, void* d_ws, int64_t ws_bytes, cudaStream_t s) {
+  const size_t esz = x_dtype == LQ_BF16 ? 2 : 4;
+  if (mode == LQ_OPEN) {
+    // step (t, l) reads x at element offset M * (t * sum_K + sum_{l' < l} K_l') and
+    // writes y at M * (t * sum_N + sum_{l' < l} N_l'); loops of a layer are
+    // independent, so up to loops_per_launch of them share one launch
+    int64_t sum_k = 0, sum_n = 0;
+    for (int l = 0; l < L; ++l) {
+      sum_k += layers[l]->wq->K;
+      sum_n += layers[l]->wq->N;
+    }
+    int nb_all = kMaxLoopsPerLaunch;
+    for (int l = 0; l < L; ++l) nb_all = std::min(nb_all, loops_per_launch(layers[l], M, T, ws_bytes));
+    bool first = true;
+    for (int t = 0; t < T; t += nb_all) {
+      const int nb = std::min(nb_all, T - t);
+      int64_t k_before = 0, n_before = 0;
+      for (int l = 0; l < L; ++l) {
+        const lq_layer* ly = layers[l];
+        const char* xin = (const char*)d_x + (size_t)(M * (t * sum_k + k_before)) * esz;
+        float* yout = d_y + M * (t * sum_n + n_before);
+        lq_status st = enqueue_linear(xin, x_dtype, M, ly, t, yout, d_ws, s, !first, true, nb,
+                                      M * sum_k, M * sum_n);
+        if (st != LQ_OK) return st;
+        first = false;
+        k_before += ly->wq->K;
+        n_before += ly->wq->N;
+      }
+    }
+    return LQ_OK;
+  }
   float* ycur = d_y;
   const float* prev_y = nullptr;
   for (int t = 0; t < T; ++t) {
     for (int l = 0; l < L; ++l) {
       const lq_layer* ly = layers[l];
-      const void* xin;
-      int32_t dt;
-      if (mode == LQ_OPEN) {
-        xin = xcur;
-        dt = x_dtype;
-        xcur += M * ly->wq->K * (x_dtype == LQ_BF16 ? 2 : 4);
-      } else {
-        xin = prev_y ? (const void*)prev_y : d_x;
-        dt = prev_y ? LQ_F32 : x_dtype;
-      }
-      lq_status st = enqueue_linear(xin, dt, M, ly, t, ycur, d_ws, s);
+      const void* xin = prev_y ? (const void*)prev_y : d_x;
+      const int32_t dt = prev_y ? LQ_F32 : x_dtype;
+      // every linear after the first overlaps its predecessor; its input is
+      // the previous output, written inside the sequence
+      const bool first = prev_y == nullptr;
+      lq_status st = enqueue_linear(xin, dt, M, ly, t, ycur, d_ws, s, !first, first);
       if (st != LQ_OK) return st;
       prev_y = ycur;
       ycur += M * ly->wq->N;
@@ -676,7 +756,7 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
     probing = g_probe.on;
   }
   if (cap != cudaStreamCaptureStatusNone || probing)
-    return enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, s);
+    return enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, ws_bytes, s);
 
   GraphKey key;
   key.x = d_x;
@@ -704,7 +784,7 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
     }
     if ((e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal)) != cudaSuccess)
       return cuda_error(e, "begin capture");
-    st = enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, cs);
+    st = enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, ws_bytes, cs);
     cudaGraph_t g = nullptr;
     e = cudaStreamEndCapture(cs, &g);
     if (st != LQ_OK) {

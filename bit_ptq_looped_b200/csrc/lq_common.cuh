@@ -19,7 +19,21 @@ constexpr int kGroup = 32;
 enum OperandFormat : int {
   kOpInt8 = 0,  // two's-complement int8 codes (tcgen05 kind::i8, GEMV)
   kOpE4M3 = 1,  // the same integer codes (|q| <= 7) encoded as FP8 E4M3 (kind::f8f6f4)
+  kOpGemvAct = 2,  // int8 codes in the decode GEMV's word order, plus per-group code sums
 };
+
+// Decode GEMV activation layout (written by the quantizer with kOpGemvAct,
+// read by k_group_gemv).  For row m and group g the 32 int8 codes c0..c31
+// become eight 32-bit words: e_i = (c_{8i}, c_{8i+2}, c_{8i+4}, c_{8i+6}) and
+// o_i = (c_{8i+1}, c_{8i+3}, c_{8i+5}, c_{8i+7}), low byte first, which line
+// up with the low and high nibbles of packed weight word i.  Half h of the
+// group holds {e_2h, o_2h, e_2h+1, o_2h+1} as one 16-byte vector at vector
+// index (m * 2 + h) * G + g, so the lanes of a warp that own consecutive
+// groups read consecutive vectors.  The group's code sum goes to
+// asum[m * G + g].
+__host__ __device__ inline int64_t gemv_act_vec_index(int64_t m, int64_t h, int64_t g, int64_t G) {
+  return (m * 2 + h) * G + g;
+}
 
 // ---------------------------------------------------------------------------
 // host-side error text (thread-local), defined in lq_api.cu
@@ -42,6 +56,58 @@ __device__ __forceinline__ uint32_t encode_e4m3_int(int q) {
 
 __device__ __forceinline__ uint32_t encode_code_byte(int q, int opf) {
   return opf == kOpE4M3 ? encode_e4m3_int(q) : ((uint32_t)q & 0xFFu);
+}
+
+// Several loops of one layer in one quantize launch (open mode): launch row r
+// belongs to loop segment j = r / seg_rows, reads its input row from
+// x + j * x_stride + (r - j * seg_rows) * K (elements) and uses clip c[j].
+// A single loop is seg_rows >= M, c[0] its clip.
+constexpr int kMaxLoopsPerLaunch = 8;
+struct LoopSegs {
+  int64_t seg_rows;
+  int64_t x_stride;
+  float c[kMaxLoopsPerLaunch];
+};
+inline LoopSegs one_loop(float c) {
+  LoopSegs s{};
+  s.seg_rows = INT64_MAX;
+  s.x_stride = 0;
+  s.c[0] = c;
+  return s;
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch (PTX griddepcontrol).  A kernel launched with
+// programmatic stream serialization may start while the previous kernel of
+// the stream is still running, as soon as every block of that kernel has
+// executed pdl_trigger (or exited).  pdl_wait blocks the calling thread until
+// the previous kernel has completed and its memory writes are visible; in a
+// kernel launched without the attribute it returns at once.  Every kernel of
+// the library calls pdl_wait before its first global write and before reading
+// anything an earlier kernel of the same sequence wrote, so completion is
+// ordered along the stream exactly as without the attribute.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kernel` on stream s, with programmatic stream serialization when
+// `pdl` is set (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // ---------------------------------------------------------------------------
@@ -248,9 +314,16 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
 int num_sms();
 
 // quantize / rotate (lq_quant.cu)
+// pdl: launch with programmatic stream serialization; x_early: x was written
+// before the sequence started, so it may be read before pdl_wait.  asum: the
+// per-group code sums of the kOpGemvAct layout (else unused).
+// segs: the clip (and, for the rotating path, the loop segments) of the rows;
+// without P1 the launch must be a single loop.
 cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, const float* P1,
-                            int a, const float* P2, int b, float c, int bits, int8_t* codes8,
-                            int opf, uint8_t* codes4, float* scales, cudaStream_t s);
+                            int a, const float* P2, int b, const LoopSegs& segs, int bits,
+                            int8_t* codes8, int opf, uint8_t* codes4, float* scales,
+                            cudaStream_t s, bool pdl = false, bool x_early = true,
+                            int* asum = nullptr);
 cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const float* Q1, int a,
                                 const float* Q2, int b, float* out, cudaStream_t s);
 cudaError_t launch_codes4_to_operand(const uint8_t* codes4, int64_t n_bytes, int opf,
@@ -259,17 +332,20 @@ cudaError_t launch_transpose_f32(const float* in, int64_t rows, int64_t cols, fl
                                  cudaStream_t s);
 size_t rotate_smem_bytes(int a, int b, int* rows_per_block);
 
-// GEMM (lq_gemm.cu)
+// GEMM (lq_gemm.cu).  Output row r goes to y + j * y_stride + (r - j * y_seg_rows) * N,
+// j = r / y_seg_rows (one segment when y_seg_rows >= M).
 cudaError_t launch_group_gemm(const uint8_t* A, const float* sa, const uint8_t* B,
                               const float* sw_t, float* y, int64_t M, int64_t N, int64_t K,
-                              int opf, cudaStream_t s, const char** why);
+                              int opf, cudaStream_t s, const char** why, bool pdl = false,
+                              int64_t y_seg_rows = INT64_MAX, int64_t y_stride = 0);
 lq_status read_and_clear_device_status(cudaStream_t s);
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
 
 // GEMV (lq_gemv.cu)
-cudaError_t launch_group_gemv(const int8_t* qa, const float* sa, const uint8_t* w4,
-                              const float* sw, float* y, int64_t M, int64_t N, int64_t K,
-                              cudaStream_t s);
+// qa: activation codes in the kOpGemvAct layout, asum their group sums
+cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa,
+                              const uint8_t* w4, const float* sw, float* y, int64_t M, int64_t N,
+                              int64_t K, cudaStream_t s, bool pdl = false);
 constexpr int kGemvMaxM = 16;
 
 }  // namespace lq

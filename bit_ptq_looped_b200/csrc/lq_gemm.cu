@@ -119,7 +119,8 @@ template <int kKindI8>
 __global__ void __launch_bounds__(THREADS, 1)
     k_group_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSW,
-                 float* __restrict__ y, int M, int N, int G) {
+                 float* __restrict__ y, int M, int N, int G, int64_t y_seg_rows,
+                 int64_t y_stride) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
 
+  pdl_trigger();  // the next kernel of the sequence may start its own prologue
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == WARP_TMA) {
     if (lane == 0) {
+      pdl_wait();  // A and its steps come from the previous kernel
       int issued = 0;
       for (int kb = 0; kb < n_kb; ++kb) {
         const int st = kb % STAGES;
@@ -236,6 +239,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     float2 acc[EPI_COLS / 2];
 #pragma unroll
     for (int i = 0; i < EPI_COLS / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+    pdl_wait();  // y may be read by a kernel before the previous one
     bool ok = true;
     for (int gi = 0; gi < G && ok; gi += 2) {
       const int kb = gi / GPS, j = gi % GPS, st = kb % STAGES;
@@ -289,7 +293,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     const int gm = m0 + row;
     if (ok && gm < M) {
-      float* yr = y + (size_t)gm * N + n0 + col0;
+      const int64_t j = gm / y_seg_rows;  // loop segment of this row
+      float* yr = y + j * y_stride + (gm - j * y_seg_rows) * (int64_t)N + n0 + col0;
 #pragma unroll
       for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
         if (n0 + col0 + 4 * c4 < N)
@@ -342,7 +347,7 @@ bool make_map_2d(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, uint
 template <int kKindI8>
 cudaError_t launch_impl(const uint8_t* A, const float* sa, const uint8_t* B, const float* sw_t,
                         float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
-                        const char** why) {
+                        const char** why, bool pdl, int64_t y_seg_rows, int64_t y_stride) {
   const int64_t G = K / kGroup;
   CUtensorMap mA, mB, mSA, mSW;
   if (!make_map_2d(&mA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, BK, BM,
@@ -367,18 +372,21 @@ cudaError_t launch_impl(const uint8_t* A, const float* sa, const uint8_t* B, con
     attr_set_mask |= 1ull << (dev & 63);
   }
   dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-  k<<<grid, THREADS, SMEM_BYTES, s>>>(mA, mB, mSA, mSW, y, (int)M, (int)N, (int)G);
-  return cudaGetLastError();
+  return launch_kernel(k, grid, dim3(THREADS), SMEM_BYTES, s, pdl, mA, mB, mSA, mSW, y, (int)M,
+                       (int)N, (int)G, y_seg_rows, y_stride);
 }
 
 }  // namespace
 
 cudaError_t launch_group_gemm(const uint8_t* A, const float* sa, const uint8_t* B,
                               const float* sw_t, float* y, int64_t M, int64_t N, int64_t K,
-                              int opf, cudaStream_t s, const char** why) {
+                              int opf, cudaStream_t s, const char** why, bool pdl,
+                              int64_t y_seg_rows, int64_t y_stride) {
   if (M == 0 || N == 0) return cudaSuccess;
-  if (opf == kOpE4M3) return launch_impl<0>(A, sa, B, sw_t, y, M, N, K, s, why);
-  return launch_impl<1>(A, sa, B, sw_t, y, M, N, K, s, why);
+  if (y_seg_rows <= 0) return cudaErrorInvalidValue;
+  if (opf == kOpE4M3)
+    return launch_impl<0>(A, sa, B, sw_t, y, M, N, K, s, why, pdl, y_seg_rows, y_stride);
+  return launch_impl<1>(A, sa, B, sw_t, y, M, N, K, s, why, pdl, y_seg_rows, y_stride);
 }
 
 namespace {

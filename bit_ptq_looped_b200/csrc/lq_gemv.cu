@@ -4,17 +4,24 @@
 //
 // Same arithmetic as the tensor-core GEMM, for the decode regime where each
 // loop reads the packed 4-bit weights once and the activation is a handful of
-// rows.  A warp walks weight rows n; lane L owns groups L, L+32, ...: one
-// 16-byte load brings the 32 packed codes of a group, one 4-byte load its
-// step.  The activation codes of all M rows sit in shared memory, rearranged
-// so a group's even and odd elements form separate 32-bit words that match
-// the low and high nibbles of the packed weights.
+// rows.  Warp w of the grid owns weight rows w, w + W, w + 2W, ... (W warps in
+// the grid); lane L owns groups L, L + 32, ... of each row: one 16-byte load
+// brings the 32 packed codes of a group, one 4-byte load its step.  The
+// activation codes of all M rows arrive in the kOpGemvAct layout (even and odd
+// codes of a group in separate 32-bit words that match the low and high
+// nibbles of the packed weights) and are copied to shared memory as they are.
 //
 // Integer dot: weight nibble v (two's complement q_w) is read as v ^ 8 =
 // q_w + 8 in [1, 15], so dp4a(unsigned weights, signed activations) gives
-// sum (q_w + 8) q_a; subtracting 8 * sum q_a (precomputed per row and group)
-// leaves the exact sum q_w q_a.
+// sum (q_w + 8) q_a; subtracting 8 * sum q_a (the group sums the quantizer
+// wrote) leaves the exact sum q_w q_a.
+//
+// The first batch of weight rows is loaded into registers before pdl_wait, so
+// under programmatic dependent launch the weight stream of this launch
+// overlaps the quantizer that produces its activation.
 #include <algorithm>
+#include <mutex>
+#include <unordered_map>
 
 #include "lq_common.cuh"
 
@@ -23,7 +30,6 @@ namespace {
 
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kGemvGroupsPerLane = 8;  // K <= 8192: each lane owns at most 8 groups of a row
 
 __device__ __forceinline__ int dp4a_us(uint32_t a_unsigned, uint32_t b_signed, int c) {
   int d;
@@ -31,174 +37,183 @@ __device__ __forceinline__ int dp4a_us(uint32_t a_unsigned, uint32_t b_signed, i
   return d;
 }
 
-// Warp w of block x owns weight rows n0 .. n0 + RPW - 1, n0 = (x * 8 + w) * RPW;
-// lane L owns groups L, L + 32, ... of each row.  Every weight load of the
-// warp is issued at entry, before the activation is staged in shared memory,
-// so the weight stream overlaps the staging.
-// shared layout: act[m][i][g] = uint2{even word, odd word} of word i (0..3) of
-// group g of row m;  asum[m][g] = sum of the group's codes;  ssa[m][g] steps.
-template <int MB, int RPW>
+// MB: activation rows handled (M <= MB); GPL: group slots per lane (G <= 32 * GPL);
+// RPW: weight rows per warp per batch.
+// shared layout: act vectors [(m * 2 + h) * G + g] (uint4), then asum[M * G], ssa[M * G].
+template <int MB, int GPL, int RPW>
 __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
-    const int8_t* __restrict__ qa, const float* __restrict__ sa, const uint8_t* __restrict__ w4,
-    const float* __restrict__ sw, float* __restrict__ y, int M, int N, int K) {
+    const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
+    const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
+    int N, int K) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
   const int G = K / kGroup;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = (blockIdx.x * kGemvWarps + warp) * RPW;
-  const int rowstride = K / 2;  // bytes per packed weight row
+  const int gw = blockIdx.x * kGemvWarps + warp;       // this warp's index in the grid
+  const int W = gridDim.x * kGemvWarps;                 // warps in the grid
+  const size_t rowstride = (size_t)K / 2;               // bytes per packed weight row
 
-  // ---- weight stream of this warp (registers)
-  uint4 wv[RPW][kGemvGroupsPerLane];
-  float swv[RPW][kGemvGroupsPerLane];
+  uint4 wv[RPW][GPL];
+  float swv[RPW][GPL];
+  auto load_batch = [&](int j0) {  // rows gw + (j0 + r) * W, r < RPW
 #pragma unroll
-  for (int r = 0; r < RPW; ++r) {
-    const int n = min(n0 + r, N - 1);
+    for (int r = 0; r < RPW; ++r) {
+      const int n = gw + (j0 + r) * W;
 #pragma unroll
-    for (int gi = 0; gi < kGemvGroupsPerLane; ++gi) {
-      const int g = lane + 32 * gi;
-      if (g < G) {
-        wv[r][gi] = __ldg(reinterpret_cast<const uint4*>(w4 + (size_t)n * rowstride) + g);
-        swv[r][gi] = __ldg(sw + (size_t)n * G + g);
-      } else {
-        wv[r][gi] = make_uint4(0, 0, 0, 0);
-        swv[r][gi] = 0.f;
-      }
-    }
-  }
-
-  // ---- stage the activation: one thread per 8-code chunk, 4 chunks per group
-  uint2* act = reinterpret_cast<uint2*>(smem_raw);                        // M*4*G
-  int* asum = reinterpret_cast<int*>(act + (size_t)M * 4 * G);           // M*G
-  float* ssa = reinterpret_cast<float*>(asum + (size_t)M * G);           // M*G
-  const int n_chunks = M * K / 8;
-  constexpr int kU = 4;  // staging loads in flight per thread
-  for (int base = 0; base < n_chunks; base += kU * kGemvThreads) {
-    uint2 raw[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int ch = base + u * kGemvThreads + threadIdx.x;
-      raw[u] = ch < n_chunks ? __ldg(reinterpret_cast<const uint2*>(qa) + ch) : make_uint2(0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int ch = base + u * kGemvThreads + threadIdx.x;
-      // n_chunks is a multiple of 4, so the 4 lanes of a group agree on validity
-      const bool valid = ch < n_chunks;
-      // bytes c0..c7 -> even word (c0,c2,c4,c6), odd word (c1,c3,c5,c7)
-      const uint32_t ev = __byte_perm(raw[u].x, raw[u].y, 0x6420);
-      const uint32_t od = __byte_perm(raw[u].x, raw[u].y, 0x7531);
-      int sum = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        sum += (int)(int8_t)((raw[u].x >> (8 * i)) & 0xFF) +
-               (int)(int8_t)((raw[u].y >> (8 * i)) & 0xFF);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-      if (valid) {
-        const int m = ch / (K / 8);
-        const int rem = ch - m * (K / 8);
-        const int g = rem >> 2, i = rem & 3;
-        act[((size_t)m * 4 + i) * G + g] = make_uint2(ev, od);
-        if (i == 0) {
-          asum[m * G + g] = sum;
-          ssa[m * G + g] = sa[(size_t)m * G + g];
+      for (int gi = 0; gi < GPL; ++gi) {
+        const int g = lane + 32 * gi;
+        if (n < N && g < G) {
+          wv[r][gi] = __ldg(reinterpret_cast<const uint4*>(w4 + (size_t)n * rowstride) + g);
+          swv[r][gi] = __ldg(sw + (size_t)n * G + g);
+        } else {
+          wv[r][gi] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+          swv[r][gi] = 0.f;
         }
       }
     }
+  };
+  load_batch(0);
+
+  // ---- the activation: written by the previous kernel of the sequence
+  pdl_wait();
+  uint4* act = reinterpret_cast<uint4*>(smem_raw);                   // M * 2 * G vectors
+  int* asum = reinterpret_cast<int*>(act + (size_t)M * 2 * G);       // M * G
+  float* ssa = reinterpret_cast<float*>(asum + (size_t)M * G);       // M * G
+  {
+    const int n_vec = M * 2 * G;
+    const uint4* src = reinterpret_cast<const uint4*>(qa);
+    for (int i = threadIdx.x; i < n_vec; i += kGemvThreads) act[i] = __ldg(src + i);
+    for (int i = threadIdx.x; i < M * G; i += kGemvThreads) {
+      asum[i] = __ldg(asum_g + i);
+      ssa[i] = __ldg(sa + i);
+    }
   }
   __syncthreads();
-  if (n0 >= N) return;
 
-  // ---- integer dots: weight nibble v read as v ^ 8 = q_w + 8 in [1, 15]
-  float part[RPW][MB];
+  for (int j0 = 0; gw + j0 * W < N; j0 += RPW) {
+    if (j0 > 0) load_batch(j0);
+    float part[RPW][MB];
 #pragma unroll
-  for (int r = 0; r < RPW; ++r)
+    for (int r = 0; r < RPW; ++r)
 #pragma unroll
-    for (int m = 0; m < MB; ++m) part[r][m] = 0.f;
+      for (int m = 0; m < MB; ++m) part[r][m] = 0.f;
 #pragma unroll
-  for (int gi = 0; gi < kGemvGroupsPerLane; ++gi) {
-    const int g = lane + 32 * gi;
-    if (g < G) {
+    for (int gi = 0; gi < GPL; ++gi) {
+      const int g = lane + 32 * gi;
+      if (g < G) {
+        uint32_t lo[RPW][4], hi[RPW][4];
 #pragma unroll
-      for (int r = 0; r < RPW; ++r) {
-        const uint4 w = wv[r][gi];
-        const uint32_t wu[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u,
-                                w.w ^ 0x88888888u};
+        for (int r = 0; r < RPW; ++r) {
+          const uint32_t wu[4] = {wv[r][gi].x ^ 0x88888888u, wv[r][gi].y ^ 0x88888888u,
+                                  wv[r][gi].z ^ 0x88888888u, wv[r][gi].w ^ 0x88888888u};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            lo[r][i] = wu[i] & 0x0F0F0F0Fu;
+            hi[r][i] = (wu[i] >> 4) & 0x0F0F0F0Fu;
+          }
+        }
 #pragma unroll
         for (int m = 0; m < MB; ++m) {
           if (m < M) {
-            int d = 0;
+            const uint4 a0 = act[gemv_act_vec_index(m, 0, g, G)];
+            const uint4 a1 = act[gemv_act_vec_index(m, 1, g, G)];
+            const int corr = 8 * asum[m * G + g];
+            const float sam = ssa[m * G + g];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint2 av = act[((size_t)m * 4 + i) * G + g];
-              d = dp4a_us(wu[i] & 0x0F0F0F0Fu, av.x, d);
-              d = dp4a_us((wu[i] >> 4) & 0x0F0F0F0Fu, av.y, d);
+            for (int r = 0; r < RPW; ++r) {
+              int d = dp4a_us(lo[r][0], a0.x, 0);
+              d = dp4a_us(hi[r][0], a0.y, d);
+              d = dp4a_us(lo[r][1], a0.z, d);
+              d = dp4a_us(hi[r][1], a0.w, d);
+              d = dp4a_us(lo[r][2], a1.x, d);
+              d = dp4a_us(hi[r][2], a1.y, d);
+              d = dp4a_us(lo[r][3], a1.z, d);
+              d = dp4a_us(hi[r][3], a1.w, d);
+              part[r][m] = fmaf(sam * swv[r][gi], (float)(d - corr), part[r][m]);
             }
-            d -= 8 * asum[m * G + g];
-            part[r][m] = fmaf(ssa[m * G + g] * swv[r][gi], (float)d, part[r][m]);
           }
         }
       }
     }
-  }
-#pragma unroll
-  for (int r = 0; r < RPW; ++r) {
-#pragma unroll
-    for (int m = 0; m < MB; ++m) {
-      float v = part[r][m];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-      part[r][m] = v;
-    }
-  }
-  if (lane == 0) {
 #pragma unroll
     for (int r = 0; r < RPW; ++r) {
-      const int n = n0 + r;
-      if (n < N) {
 #pragma unroll
-        for (int m = 0; m < MB; ++m)
-          if (m < M) y[(size_t)m * N + n] = part[r][m];
+      for (int m = 0; m < MB; ++m) {
+        float v = part[r][m];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        part[r][m] = v;
       }
+    }
+    // lane (r * MB + m) % 32 writes y[m, n_r]
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const int n = gw + (j0 + r) * W;
+#pragma unroll
+      for (int m = 0; m < MB; ++m)
+        if (lane == ((r * MB + m) & 31) && m < M && n < N) y[(size_t)m * N + n] = part[r][m];
     }
   }
 }
 
-template <int MB, int RPW>
-cudaError_t launch_mb(const int8_t* qa, const float* sa, const uint8_t* w4, const float* sw,
-                      float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
-  const int64_t G = K / kGroup;
-  const size_t smem = (size_t)M * 4 * G * 8 + (size_t)M * G * 8;
-  auto* k = k_group_gemv<MB, RPW>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
+size_t gemv_smem_bytes(int64_t M, int64_t G) { return (size_t)M * G * (32 + 8); }
+
+template <int MB, int GPL, int RPW>
+cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
+                       const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                       bool pdl) {
+  const size_t smem = gemv_smem_bytes(M, K / kGroup);
+  auto* k = k_group_gemv<MB, GPL, RPW>;
+  // resident blocks per SM for this instantiation and shared-memory size
+  static std::mutex mu;
+  static std::unordered_map<size_t, int> per_sm_cache;
+  int per_sm = 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = per_sm_cache.find(smem);
+    if (it == per_sm_cache.end()) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)std::max<size_t>(smem, 1));
+      if (e != cudaSuccess) return e;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemvThreads, smem);
+      if (e != cudaSuccess) return e;
+      if (per_sm < 1) return cudaErrorInvalidConfiguration;
+      per_sm_cache.emplace(smem, per_sm);
+    } else {
+      per_sm = it->second;
+    }
   }
+  // enough warps for one batch of RPW rows each, capped at one resident wave
   const int64_t warps_needed = (N + RPW - 1) / RPW;
-  const int64_t blocks = (warps_needed + kGemvWarps - 1) / kGemvWarps;
-  k<<<(unsigned)blocks, kGemvThreads, smem, s>>>(qa, sa, w4, sw, y, (int)M, (int)N, (int)K);
-  return cudaGetLastError();
+  const int64_t want = (warps_needed + kGemvWarps - 1) / kGemvWarps;
+  const int64_t blocks = std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
+  return launch_kernel(k, dim3((unsigned)blocks), dim3(kGemvThreads), smem, s, pdl, qa, asum, sa,
+                       w4, sw, y, (int)M, (int)N, (int)K);
 }
 
 template <int MB>
-cudaError_t launch_rows(const int8_t* qa, const float* sa, const uint8_t* w4, const float* sw,
-                        float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
-  // two rows per warp once there are enough rows to fill the GPU twice over
-  if (N >= 4096) return launch_mb<MB, 2>(qa, sa, w4, sw, y, M, N, K, s);
-  return launch_mb<MB, 1>(qa, sa, w4, sw, y, M, N, K, s);
+cudaError_t launch_mb(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
+                      const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                      bool pdl) {
+  const int64_t G = K / kGroup;
+  if (G > 128) return launch_cfg<MB, 8, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  if (G > 64) return launch_cfg<MB, 4, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  // three rows per warp once that still gives every SM one and a half blocks
+  if (N >= (int64_t)num_sms() * kGemvWarps * 3 * 3 / 2)
+    return launch_cfg<MB, 2, 3>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_cfg<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
 }  // namespace
 
-cudaError_t launch_group_gemv(const int8_t* qa, const float* sa, const uint8_t* w4,
-                              const float* sw, float* y, int64_t M, int64_t N, int64_t K,
-                              cudaStream_t s) {
+cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa,
+                              const uint8_t* w4, const float* sw, float* y, int64_t M, int64_t N,
+                              int64_t K, cudaStream_t s, bool pdl) {
   if (M == 0 || N == 0) return cudaSuccess;
-  if (K > (int64_t)kGroup * 32 * kGemvGroupsPerLane) return cudaErrorInvalidValue;
-  if (M <= 1) return launch_rows<1>(qa, sa, w4, sw, y, M, N, K, s);
-  if (M <= 4) return launch_rows<4>(qa, sa, w4, sw, y, M, N, K, s);
-  return launch_rows<16>(qa, sa, w4, sw, y, M, N, K, s);
+  if (K > (int64_t)kGroup * 32 * 8 || M > kGemvMaxM) return cudaErrorInvalidValue;
+  if (M <= 1) return launch_mb<1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  if (M <= 4) return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_mb<16>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
 }  // namespace lq

@@ -103,11 +103,27 @@ __device__ __forceinline__ uint32_t e4m3_byte(uint32_t qb) {
   return byte | (q < 0 ? 0x80u : 0u);
 }
 
-// Write one thread's 8 codes (and its group's step from lane 4j).
+// Sum of the 32 codes of the group whose 8 codes this thread holds (the 4
+// lanes 4j..4j+3 of the group all get it).  Every lane of the warp must call it.
+__device__ __forceinline__ int group_code_sum(const uint32_t (&qb)[8]) {
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sum += (int)(int8_t)(qb[i] & 0xFFu);
+  sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+  sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+  return sum;
+}
+
+// Write one thread's 8 codes (and its group's step from lane 4j).  chunk is
+// the index of the 8-code chunk in the M x K activation.  kGemvAct selects the
+// decode GEMV layout (opf == kOpGemvAct): G is the number of groups per row
+// and gsum the group's code sum.
+template <bool kGemvAct>
 __device__ __forceinline__ void store_codes(const uint32_t (&qb)[8], float s, int64_t chunk,
                                             int8_t* __restrict__ codes8, int opf,
                                             uint8_t* __restrict__ codes4,
-                                            float* __restrict__ scales) {
+                                            float* __restrict__ scales, int G = 0, int gsum = 0,
+                                            int* __restrict__ asum = nullptr) {
   if (codes8) {
     uint2 w;
     if (opf == kOpE4M3) {
@@ -117,7 +133,19 @@ __device__ __forceinline__ void store_codes(const uint32_t (&qb)[8], float s, in
       w.x = pack_bytes4(qb[0], qb[1], qb[2], qb[3]);
       w.y = pack_bytes4(qb[4], qb[5], qb[6], qb[7]);
     }
-    reinterpret_cast<uint2*>(codes8)[chunk] = w;
+    if (kGemvAct) {
+      // chunk = (m * G + g) * 4 + i: words e_i, o_i of group g of row m
+      const int64_t grp = chunk >> 2;
+      const int i = (int)(chunk & 3);
+      const int64_t m = grp / G, g = grp - m * G;
+      const uint32_t ev = __byte_perm(w.x, w.y, 0x6420), od = __byte_perm(w.x, w.y, 0x7531);
+      uint2* dst = reinterpret_cast<uint2*>(codes8) + 2 * gemv_act_vec_index(m, i >> 1, g, G) +
+                   (i & 1);
+      *dst = make_uint2(ev, od);
+      if (i == 0) asum[grp] = gsum;
+    } else {
+      reinterpret_cast<uint2*>(codes8)[chunk] = w;
+    }
   }
   if (codes4) {
     uint32_t p = 0;
@@ -135,16 +163,20 @@ struct FastDiv {
   __device__ __forceinline__ uint32_t div(uint32_t n) const { return d == 1u ? n : __umulhi(n, m); }
 };
 
-template <typename Tin>
+template <typename Tin, bool kGemvAct>
 __global__ void __launch_bounds__(kThreads) k_quant_only(const Tin* __restrict__ x,
                                                          int64_t n_chunks, float c, int qmax,
                                                          int8_t* __restrict__ codes8, int opf,
                                                          uint8_t* __restrict__ codes4,
-                                                         float* __restrict__ scales) {
+                                                         float* __restrict__ scales, int G,
+                                                         int* __restrict__ asum, int x_early) {
+  pdl_trigger();
+  if (!x_early) pdl_wait();
   // Two 8-element chunks per thread per step (blockDim apart) keep more loads
   // in flight.  n_chunks is a multiple of 4 and every bound below is
   // warp-uniform, so the 4 lanes of a group are all valid or all invalid.
   const int64_t stride = (int64_t)gridDim.x * (2 * kThreads);
+  bool waited = !x_early;
   for (int64_t base = (int64_t)blockIdx.x * (2 * kThreads); base < n_chunks; base += stride) {
     const int64_t ch0 = base + threadIdx.x, ch1 = ch0 + kThreads;
     const bool v0 = ch0 < n_chunks, v1 = ch1 < n_chunks;
@@ -162,8 +194,17 @@ __global__ void __launch_bounds__(kThreads) k_quant_only(const Tin* __restrict__
     uint32_t q0[8], q1[8];
     const float s0 = quant_group8(a0, c, qmax, q0);
     const float s1 = quant_group8(a1, c, qmax, q1);
-    if (v0) store_codes(q0, s0, ch0, codes8, opf, codes4, scales);
-    if (v1) store_codes(q1, s1, ch1, codes8, opf, codes4, scales);
+    int gs0 = 0, gs1 = 0;
+    if (kGemvAct) {
+      gs0 = group_code_sum(q0);
+      gs1 = group_code_sum(q1);
+    }
+    if (!waited) {  // the previous kernel may still read the output buffers
+      pdl_wait();
+      waited = true;
+    }
+    if (v0) store_codes<kGemvAct>(q0, s0, ch0, codes8, opf, codes4, scales, G, gs0, asum);
+    if (v1) store_codes<kGemvAct>(q1, s1, ch1, codes8, opf, codes4, scales, G, gs1, asum);
   }
 }
 
@@ -261,10 +302,14 @@ constexpr int kRotTM = 2, kRotTN = 4;  // warp task: 16 x 32 outputs
 template <typename Tin, bool kStoreF32>
 __global__ void __launch_bounds__(kThreads) k_rotate_quant(
     const Tin* __restrict__ x, int64_t M, int K, const float* __restrict__ P1, int a,
-    const float* __restrict__ P2, int b, int R, float c, int qmax, int8_t* __restrict__ codes8,
+    const float* __restrict__ P2, int b, int R, const LoopSegs segs, int qmax,
+    int8_t* __restrict__ codes8,
     int opf, uint8_t* __restrict__ codes4, float* __restrict__ scales,
-    float* __restrict__ out_f32) {
+    float* __restrict__ out_f32, int* __restrict__ asum, int x_early) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  if (!x_early) pdl_wait();
+  bool waited = !x_early;
   const RotLayout L = rot_layout(a, b, R);
   double* sm = reinterpret_cast<double*>(smem_raw);
   double* P2T = sm;
@@ -272,20 +317,60 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
   double* YT = sm + L.off_yt;
   float* X = reinterpret_cast<float*>(sm + L.off_x);
   float* Z = X;  // (R*a) rows of pitch ldz floats, written after stage 1
+  // per row of the tile: input offset (elements; read before the stage-1
+  // barrier) and the loop's clip (read in the epilogue, so kept per tile parity)
+  __shared__ int64_t row_off[16];
+  __shared__ float row_c[2][16];
 
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr int kWarps = kThreads / 32;
-  for (int e = tid; e < b * b; e += kThreads) {
-    const int q = e / b, j = e - q * b;
-    P2T[(size_t)j * L.ldb + q] = (double)P2[e];
-  }
-  for (int e = tid; e < a * a; e += kThreads) {
-    const int p = e / a, i = e - p * a;
-    P1T[(size_t)i * L.lda + p] = (double)P1[e];
-  }
-
   const int row_chunks = K >> 3;
   const FastDiv fd_rowc((uint32_t)row_chunks), fd_b((uint32_t)b), fd_a((uint32_t)a);
+
+  // ---- prologue: the first tile's input and the factors are loaded with all
+  // loads of a thread in flight at once (one memory round trip, not one per
+  // element: for a few rows this latency is most of the kernel's time)
+  constexpr int kXU = 2, kFU = 24;
+  const int64_t m_first = (int64_t)blockIdx.x * R;
+  const bool x_pre = x_early && R * row_chunks <= kXU * kThreads;
+  float xr[kXU][8];
+  if (x_pre) {
+#pragma unroll
+    for (int u = 0; u < kXU; ++u) {
+      const int ch = u * kThreads + tid;
+      const int r = (int)fd_rowc.div((uint32_t)ch);
+      if (ch < R * row_chunks && m_first + r < M) {
+        const int64_t gr = m_first + r, j = gr / segs.seg_rows;
+        load8(x + j * segs.x_stride + (gr - j * segs.seg_rows) * K, ch - r * row_chunks, xr[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[u][e] = 0.f;
+      }
+    }
+  }
+  {
+    const int n2 = b * b, nf = n2 + a * a;
+    for (int base = 0; base < nf; base += kFU * kThreads) {
+      float v[kFU];
+#pragma unroll
+      for (int u = 0; u < kFU; ++u) {
+        const int e = base + u * kThreads + tid;
+        v[u] = e < n2 ? __ldg(P2 + e) : (e < nf ? __ldg(P1 + (e - n2)) : 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kFU; ++u) {
+        const int e = base + u * kThreads + tid;
+        if (e < n2) {  // P2T[j][q] = P2[q][j]
+          const int q = (int)fd_b.div((uint32_t)e), j = e - q * b;
+          P2T[(size_t)j * L.ldb + q] = (double)v[u];
+        } else if (e < nf) {  // P1T[i][p] = P1[p][i]
+          const int e1 = e - n2, p = (int)fd_a.div((uint32_t)e1), i = e1 - p * a;
+          P1T[(size_t)i * L.lda + p] = (double)v[u];
+        }
+      }
+    }
+  }
+
   // stage 1 tasks: (R*a/16) row pairs x ceil(b/32) column quads
   const int ct = b >> 3;
   const int s1_rt = (R * a) / (8 * kRotTM);
@@ -296,20 +381,46 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
   const int s2_tasks = R * s2_rt * s1_ctq;
   const FastDiv fd_s1ctq((uint32_t)s1_ctq), fd_s2tok((uint32_t)(s2_rt * s1_ctq));
 
-  for (int64_t m0 = (int64_t)blockIdx.x * R; m0 < M; m0 += (int64_t)gridDim.x * R) {
+  int par = 0;
+  bool first = true;
+  for (int64_t m0 = (int64_t)blockIdx.x * R; m0 < M; m0 += (int64_t)gridDim.x * R, par ^= 1) {
     const int rows = (M - m0 < (int64_t)R) ? (int)(M - m0) : R;
-    __syncthreads();  // previous Z consumed; factors staged
-    for (int ch = tid; ch < R * row_chunks; ch += kThreads) {
-      const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
-      const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
-      float* dst = X + (size_t)(r * a + i) * L.ldb + q;
-      if (r < rows) {
-        load_row_chunk8(x + (size_t)m0 * K, ch, dst);
-      } else {
-        reinterpret_cast<float4*>(dst)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        reinterpret_cast<float4*>(dst)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < rows) {
+      const int64_t r = m0 + tid, j = r / segs.seg_rows;
+      row_off[tid] = j * segs.x_stride + (r - j * segs.seg_rows) * K;
+      float cj = segs.c[0];  // static indices keep the parameter block out of local memory
+#pragma unroll
+      for (int u = 1; u < kMaxLoopsPerLaunch; ++u)
+        if (j == u) cj = segs.c[u];
+      row_c[par][tid] = cj;
+    }
+    __syncthreads();  // previous Z consumed; factors and row offsets staged
+    if (first && x_pre) {  // the prologue's registers (zeros past the last row)
+#pragma unroll
+      for (int u = 0; u < kXU; ++u) {
+        const int ch = u * kThreads + tid;
+        if (ch < R * row_chunks) {
+          const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
+          const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
+          float4* dst = reinterpret_cast<float4*>(X + (size_t)(r * a + i) * L.ldb + q);
+          dst[0] = make_float4(xr[u][0], xr[u][1], xr[u][2], xr[u][3]);
+          dst[1] = make_float4(xr[u][4], xr[u][5], xr[u][6], xr[u][7]);
+        }
+      }
+    } else {
+      for (int ch = tid; ch < R * row_chunks; ch += kThreads) {
+        const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
+        const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
+        float* dst = X + (size_t)(r * a + i) * L.ldb + q;
+        if (r < rows) {
+          load_row_chunk8(x + row_off[r], ch - r * row_chunks, dst);
+        } else {
+          reinterpret_cast<float4*>(dst)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+          reinterpret_cast<float4*>(dst)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
     }
+    first = false;
     __syncthreads();
     // ---- stage 1: Y[(r,i), j] = sum_q X[(r,i), q] P2[q, j]  -> YT[r][j][i]
     for (int task = warp; task < s1_tasks; task += kWarps) {
@@ -338,6 +449,10 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
                                     });
     }
     __syncthreads();
+    if (!waited) {  // the previous kernel may still read the output buffers
+      pdl_wait();
+      waited = true;
+    }
     // ---- epilogue: chunk ch covers elements 8*ch .. 8*ch+7 of the R-row tile
     if (kStoreF32) {
       for (int ch = tid; ch < rows * row_chunks; ch += kThreads) {
@@ -355,6 +470,7 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
         const int r = (int)fd_rowc.div((uint32_t)ch);
         const bool valid = ch < n_chunks && r < rows;
         float v[8];
+        const float c = valid ? row_c[par][r] : 1.f;
         if (valid) {
           const int k8 = (ch - r * row_chunks) * 8;
           const int i = (int)fd_b.div((uint32_t)k8), j = k8 - i * b;
@@ -369,7 +485,14 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
         }
         uint32_t q[8];
         const float s = quant_group8(v, c, qmax, q);
-        if (valid) store_codes(q, s, m0 * row_chunks + ch, codes8, opf, codes4, scales);
+        if (opf == kOpGemvAct) {
+          const int gs = group_code_sum(q);
+          if (valid)
+            store_codes<true>(q, s, m0 * row_chunks + ch, codes8, opf, codes4, scales,
+                              K / kGroup, gs, asum);
+        } else if (valid) {
+          store_codes<false>(q, s, m0 * row_chunks + ch, codes8, opf, codes4, scales);
+        }
       }
     }
   }
@@ -427,32 +550,40 @@ int num_sms() {
 }
 
 size_t rotate_smem_bytes(int a, int b, int* rows_per_block) {
-  // prefer two resident blocks per SM (<= 113 KB each), else one (<= 227 KB)
+  // prefer two resident blocks per SM (<= 112 KB each, leaving room for the
+  // static row arrays), else one (<= 226 KB)
   int best = 0;
   for (int R = 16; R >= 1; R >>= 1) {
-    if (rot_layout(a, b, R).bytes <= 113u * 1024u) { best = R; break; }
+    if (rot_layout(a, b, R).bytes <= 112u * 1024u) { best = R; break; }
   }
-  if (best == 0 && rot_layout(a, b, 1).bytes <= 227u * 1024u) best = 1;
+  if (best == 0 && rot_layout(a, b, 1).bytes <= 226u * 1024u) best = 1;
   if (rows_per_block) *rows_per_block = best;
   return best ? rot_layout(a, b, best).bytes : 0;
 }
 
 cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, const float* P1,
-                            int a, const float* P2, int b, float c, int bits, int8_t* codes8,
-                            int opf, uint8_t* codes4, float* scales, cudaStream_t s) {
+                            int a, const float* P2, int b, const LoopSegs& segs, int bits,
+                            int8_t* codes8, int opf, uint8_t* codes4, float* scales,
+                            cudaStream_t s, bool pdl, bool x_early, int* asum) {
   const int qmax = bits == 8 ? 127 : 7;
   if (M == 0) return cudaSuccess;
+  const float c = segs.c[0];
+  if (P1 == nullptr && segs.seg_rows < M) return cudaErrorInvalidValue;
+  if (opf == kOpGemvAct && (codes8 == nullptr || asum == nullptr)) return cudaErrorInvalidValue;
+  const int G = (int)(K / kGroup);
+  const int xe = x_early ? 1 : 0;
   if (P1 == nullptr) {
     const int64_t n_chunks = M * K / 8;
     const int64_t want = (n_chunks + 2 * kThreads - 1) / (2 * kThreads);
     const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * 8);
+    const bool gv = opf == kOpGemvAct;
     if (x_dtype == LQ_BF16)
-      k_quant_only<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
-          (const __nv_bfloat16*)x, n_chunks, c, qmax, codes8, opf, codes4, scales);
-    else
-      k_quant_only<float><<<grid, kThreads, 0, s>>>((const float*)x, n_chunks, c, qmax, codes8,
-                                                    opf, codes4, scales);
-    return cudaGetLastError();
+      return launch_kernel(gv ? k_quant_only<__nv_bfloat16, true> : k_quant_only<__nv_bfloat16, false>,
+                           dim3(grid), dim3(kThreads), 0, s, pdl, (const __nv_bfloat16*)x,
+                           n_chunks, c, qmax, codes8, opf, codes4, scales, G, asum, xe);
+    return launch_kernel(gv ? k_quant_only<float, true> : k_quant_only<float, false>, dim3(grid),
+                         dim3(kThreads), 0, s, pdl, (const float*)x, n_chunks, c, qmax, codes8,
+                         opf, codes4, scales, G, asum, xe);
   }
   int R = 0;
   size_t smem = rotate_smem_bytes(a, b, &R);
@@ -461,22 +592,22 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
     R = 1;
     smem = rot_layout(a, b, 1).bytes;
   }
-  const int per_sm = smem <= 113u * 1024u ? 2 : 1;
+  const int per_sm = smem <= 112u * 1024u ? 2 : 1;
   const int64_t want = (M + R - 1) / R;
   const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
   cudaError_t e;
   if (x_dtype == LQ_BF16) {
     auto* k = k_rotate_quant<__nv_bfloat16, false>;
     if ((e = set_smem(k, smem)) != cudaSuccess) return e;
-    k<<<grid, kThreads, smem, s>>>((const __nv_bfloat16*)x, M, (int)K, P1, a, P2, b, R, c, qmax,
-                                   codes8, opf, codes4, scales, nullptr);
-  } else {
-    auto* k = k_rotate_quant<float, false>;
-    if ((e = set_smem(k, smem)) != cudaSuccess) return e;
-    k<<<grid, kThreads, smem, s>>>((const float*)x, M, (int)K, P1, a, P2, b, R, c, qmax, codes8,
-                                   opf, codes4, scales, nullptr);
+    return launch_kernel(k, dim3(grid), dim3(kThreads), smem, s, pdl, (const __nv_bfloat16*)x, M,
+                         (int)K, P1, a, P2, b, R, segs, qmax, codes8, opf, codes4, scales,
+                         (float*)nullptr, asum, xe);
   }
-  return cudaGetLastError();
+  auto* k = k_rotate_quant<float, false>;
+  if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+  return launch_kernel(k, dim3(grid), dim3(kThreads), smem, s, pdl, (const float*)x, M, (int)K,
+                       P1, a, P2, b, R, segs, qmax, codes8, opf, codes4, scales, (float*)nullptr,
+                       asum, xe);
 }
 
 cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const float* Q1, int a,
@@ -489,13 +620,13 @@ cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const floa
     R = 1;
     smem = rot_layout(a, b, 1).bytes;
   }
-  const int per_sm = smem <= 113u * 1024u ? 2 : 1;
+  const int per_sm = smem <= 112u * 1024u ? 2 : 1;
   const int grid = (int)std::min<int64_t>((M + R - 1) / R, (int64_t)num_sms() * per_sm);
   auto* k = k_rotate_quant<float, true>;
   cudaError_t e = set_smem(k, smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, kThreads, smem, s>>>(x, M, (int)K, Q1, a, Q2, b, R, 1.0f, 7, nullptr, kOpInt8,
-                                 nullptr, nullptr, out);
+  k<<<grid, kThreads, smem, s>>>(x, M, (int)K, Q1, a, Q2, b, R, one_loop(1.0f), 7, nullptr,
+                                 kOpInt8, nullptr, nullptr, out, nullptr, 1);
   return cudaGetLastError();
 }
 

@@ -45,6 +45,7 @@ SIGNATURES = {
     "lq_layer_create": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _i32, _i32, _pp]),
     "lq_layer_free": (None, [_vp]),
     "lq_workspace_bytes": (_i64, [_pp, _i32, _i64]),
+    "lq_stack_workspace_bytes": (_i64, [_pp, _i32, _i64, _i32]),
     "lq_loop_linear": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
     "lq_check_device": (_i32, [_vp]),
@@ -268,8 +269,18 @@ def lq_workspace_bytes(layers: Sequence[Layer], M: int) -> int:
     return n
 
 
-def workspace(layers: Sequence[Layer], M: int, device="cuda") -> torch.Tensor:
-    n = lq_workspace_bytes(layers, M)
+def lq_stack_workspace_bytes(layers: Sequence[Layer], M: int, T: int) -> int:
+    p, keep = _layer_array(layers)
+    n = lib().lq_stack_workspace_bytes(p, len(layers), M, T)
+    if n < 0:
+        raise ValueError("invalid layers or T")
+    return n
+
+
+def workspace(layers: Sequence[Layer], M: int, device="cuda", T: Optional[int] = None) -> torch.Tensor:
+    """Workspace for M tokens; with T, the size that lets open-mode lq_loop_stack
+    run the T loops of a layer in one launch (lq_stack_workspace_bytes)."""
+    n = lq_workspace_bytes(layers, M) if T is None else lq_stack_workspace_bytes(layers, M, T)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 
@@ -293,7 +304,7 @@ def lq_loop_stack(x: torch.Tensor, layers: Sequence[Layer], T: int, mode: int = 
     if y is None:
         y = torch.empty(T * M * sum(l.N for l in layers), dtype=torch.float32, device=x.device)
     if ws is None:
-        ws = workspace(layers, M, x.device)
+        ws = workspace(layers, M, x.device, T=T if mode == LQ_OPEN else None)
     p, keep = _layer_array(layers)
     dt = _dtype_code(x) if x_dtype is None else x_dtype
     st = lib().lq_loop_stack(_dev(x, "x"), dt, M, p, len(layers), T, mode, _dev(y, "y"),

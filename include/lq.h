@@ -169,6 +169,16 @@ void lq_layer_free(lq_layer* layer);
 int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M);
 
 /*
+ * Workspace with which lq_loop_stack in LQ_OPEN mode runs up to min(T, 8)
+ * loops of each layer in one quantize and one GEMM launch (the loops of a
+ * layer are independent in open mode and share the resident weights).  Equal
+ * to lq_workspace_bytes for decode-sized M (the GEMV path runs loop by loop).
+ * Returns -1 on a null pointer or a non-positive L or T.
+ */
+int64_t lq_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M,
+                                 int32_t T);
+
+/*
  * lq_loop_linear -- one application of a shared quantized linear at loop t:
  * y = Q(x (P1 kron P2); c_t) (*) Wq, steps 1-4 above.
  *   d_x   M x K (x_dtype LQ_F32 or LQ_BF16);  d_y out M x N float32.
@@ -186,6 +196,15 @@ lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_l
  *   mode LQ_CHAIN: d_x holds one M x K_0 input; x_{t,l} is the previous
  *                  step's y (float32).  Needs N_l == K_{l+1} and N_{L-1} == K_0.
  *   d_y   out: T*L outputs ordered (t, l), each M x N_l float32.
+ *   d_ws  at least lq_workspace_bytes(layers, L, M) bytes, 256-byte aligned.
+ *         In LQ_OPEN mode a larger workspace lets one launch cover several
+ *         loops of a layer (as many as fit, at most 8;
+ *         lq_stack_workspace_bytes gives the size for min(T, 8)); results are
+ *         the same either way.
+ * Consecutive kernels of the schedule use programmatic dependent launch: a
+ * kernel starts its prologue (weight loads, rotation of inputs that exist
+ * before the call) while its predecessor finishes, and waits for it before
+ * reading its output or writing any buffer.
  * The schedule is recorded once into a CUDA graph per distinct argument set
  * and replayed (when `stream` is itself capturing, kernels are launched
  * directly into the caller's capture instead).

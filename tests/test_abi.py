@@ -108,6 +108,7 @@ def test_loop_entry_points_reject_bad_arguments(L):
     assert L.lq_loop_stack(fake, lq.LQ_F32, 4, None, 1, 4, lq.LQ_OPEN, fake, fake, 1 << 20,
                            None) == lq.LQ_ERR_ARG
     assert L.lq_workspace_bytes(None, 1, 4) == -1
+    assert L.lq_stack_workspace_bytes(None, 1, 4, 4) == -1
 
 
 def test_inverse_transpose_host_helper():

@@ -156,6 +156,51 @@ def test_loop_stack_open(wl, M):
             linear_parity(yg, xs[t][l], built[l][1], t, host(q8), host(s), built[l][0].w_flips)
 
 
+@pytest.mark.parametrize("wl,M", [(synth.MLP, 256), (synth.TINY, 64), (synth.ATTN_PROJ, 200)],
+                         ids=["mlp", "tiny", "attn_ragged"])
+def test_loop_stack_open_batching_matches_per_loop(wl, M):
+    """Open mode runs several loops of a layer per launch when the workspace
+    holds them.  Each output row goes through the same per-row arithmetic, so
+    every batch width (including a partial last batch, and M not a multiple of
+    the 128-row GEMM tile) must reproduce the one-loop-per-launch schedule bit
+    for bit."""
+    params = synth.module_params(wl)
+    layers = [make_layer(mp, wl.a_bits)[0] for mp in params]
+    xs, flat = _stack_inputs(wl, M)
+    xd = act_tensor(flat, wl.x_dtype)
+    T = wl.T
+    ref = lq.lq_loop_stack(xd, layers, T, lq.LQ_OPEN, M=M, ws=lq.workspace(layers, M))
+    for nb in (2, 3, T):
+        ws = lq.workspace(layers, M, T=nb)
+        assert ws.numel() >= lq.lq_workspace_bytes(layers, M) * (nb - 0.5)
+        y = lq.lq_loop_stack(xd, layers, T, lq.LQ_OPEN, M=M, ws=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref), f"batch of {nb} loops"
+
+
+def test_loop_stack_open_more_than_eight_loops():
+    """T = 11 loops with a full-size workspace: launches of 8 and 3 loops, each
+    loop with its own LAS clip, checked against the oracle loop by loop."""
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    (lin,) = wl.linears
+    T = 11
+    mp.las = np.random.default_rng(11).uniform(0.7, 1.0, T).astype(np.float32)
+    layer, ol = make_layer(mp, wl.a_bits)
+    M = wl.M
+    xs = [synth.loop_input(wl, lin, t, rows=np.arange(M)) for t in range(T)]
+    xd = act_tensor(np.concatenate([x.ravel() for x in xs]), wl.x_dtype)
+    ws = lq.workspace([layer], M, T=T)
+    y = host(lq.lq_loop_stack(xd, [layer], T, lq.LQ_OPEN, M=M, ws=ws))
+    torch.cuda.synchronize()
+    for t in range(T):
+        q8, _, s = lq.lq_quantize_act(act_tensor(xs[t], wl.x_dtype), dev(mp.P1), dev(mp.P2),
+                                      float(mp.las[t]), wl.a_bits)
+        torch.cuda.synchronize()
+        linear_parity(y[t * M * lin.N:(t + 1) * M * lin.N].reshape(M, lin.N), xs[t], ol, t,
+                      host(q8), host(s), layer.w_flips)
+
+
 def test_loop_stack_chain_tiny():
     """Chain mode feeds y_{t} back as x_{t+1} (T = 4 loops of one shared layer)."""
     wl = synth.TINY
