@@ -5,7 +5,12 @@
 // ("paper_specification.yaml" of the LoopQ reproduction: lq1_quantization,
 // weights and activations group-wise with group size 32, W4 with A4/A8.)
 //
-// One CTA owns a 128 x 128 tile of y.  Each 32-wide K group is exactly one
+// The kernel is persistent: one CTA per SM walks the 128 x 128 tiles of y
+// (t = blockIdx.x, + gridDim.x, ...; m-block-major order so concurrently
+// processed tiles share A rows and all of B in L2).  Barriers, TMEM and the
+// operand ring are set up once per CTA, and the pipeline runs straight across
+// tile boundaries: the tensor core starts a tile's first groups while the
+// epilogue still folds and stores the previous tile.  Each 32-wide K group is exactly one
 // tcgen05.mma instruction (K = 32 bytes for 8-bit operands), written to its
 // own TMEM accumulator, because the next group carries different scales and
 // cannot be summed into it.  Four 128-column accumulators rotate through the
@@ -31,6 +36,7 @@
 // TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "lq_common.cuh"
@@ -128,9 +134,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * BM;
   const int n_kb = G / GPS;
+  const int tiles_n = (N + BN - 1) / BN;
+  const int n_tiles = tiles_n * ((M + BM - 1) / BM);
 
   const uint32_t bar_full = base + OFF_BAR;
   const uint32_t bar_empty = bar_full + STAGES * 8;
@@ -172,56 +178,64 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == WARP_TMA) {
     if (lane == 0) {
       pdl_wait();  // A and its steps come from the previous kernel
-      int issued = 0;
-      for (int kb = 0; kb < n_kb; ++kb) {
-        const int st = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait_bounded(bar_empty + 8 * st, ph ^ 1u, abort_flag, &g_gemm_status,
-                               kWaitLimitNs))
-          break;
-        const uint32_t full = bar_full + 8 * st;
-        mbar_arrive_expect_tx(full, STAGE_TX);
-        tma_load_2d(base + OFF_A + st * A_BYTES, &tmA, full, kb * BK, m0);
-        tma_load_2d(base + OFF_B + st * B_BYTES, &tmB, full, kb * BK, n0);
-        tma_load_2d(base + OFF_SA + st * SA_BYTES, &tmSA, full, kb * GPS, m0);
-        tma_load_2d(base + OFF_SW + st * SW_BYTES, &tmSW, full, n0, kb * GPS);
-        issued = kb + 1;
+      int kbg = 0;  // k-blocks issued by this CTA over all its tiles
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+        for (int kb = 0; kb < n_kb; ++kb, ++kbg) {
+          const int st = kbg % STAGES;
+          const uint32_t ph = (uint32_t)(kbg / STAGES) & 1u;
+          if (!mbar_wait_bounded(bar_empty + 8 * st, ph ^ 1u, abort_flag, &g_gemm_status,
+                                 kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = bar_full + 8 * st;
+          mbar_arrive_expect_tx(full, STAGE_TX);
+          tma_load_2d(base + OFF_A + st * A_BYTES, &tmA, full, kb * BK, m0);
+          tma_load_2d(base + OFF_B + st * B_BYTES, &tmB, full, kb * BK, n0);
+          tma_load_2d(base + OFF_SA + st * SA_BYTES, &tmSA, full, kb * GPS, m0);
+          tma_load_2d(base + OFF_SW + st * SW_BYTES, &tmSW, full, n0, kb * GPS);
+        }
       }
       // never leave the CTA with bulk copies in flight: wait (bounded, even
       // after an abort) for the last STAGES loads to land
-      for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
+      for (int kb = max(0, kbg - STAGES); kb < kbg; ++kb)
         mbar_wait_drain(bar_full + 8 * (kb % STAGES), (uint32_t)(kb / STAGES) & 1u);
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc<kKindI8>();
-      int gi = 0;  // running group index
+      int kbg = 0, gi = 0;  // running k-block and group counters over all tiles
       bool ok = true;
-      for (int kb = 0; kb < n_kb && ok; ++kb) {
-        const int st = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait_bounded(bar_full + 8 * st, ph, abort_flag, &g_gemm_status, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t a_st = base + OFF_A + st * A_BYTES;
-        const uint32_t b_st = base + OFF_B + st * B_BYTES;
-        for (int j = 0; j < GPS; ++j, ++gi) {
-          const int buf = gi % ACC_BUFS;
-          const uint32_t aph = (uint32_t)(gi / ACC_BUFS) & 1u;
-          if (!mbar_wait_bounded(bar_acce + 8 * buf, aph ^ 1u, abort_flag, &g_gemm_status,
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < n_kb && ok; ++kb, ++kbg) {
+          const int st = kbg % STAGES;
+          const uint32_t ph = (uint32_t)(kbg / STAGES) & 1u;
+          if (!mbar_wait_bounded(bar_full + 8 * st, ph, abort_flag, &g_gemm_status,
                                  kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // one MMA per 32-wide group: advance 32 bytes inside the swizzled 128-byte rows
-          umma_ss<kKindI8>(tmem_base + (uint32_t)(buf * BN), sw128_kmajor_desc(a_st + 32u * j),
-                           sw128_kmajor_desc(b_st + 32u * j), idesc, 0u);
-          umma_commit(bar_accf + 8 * buf);
+          const uint32_t a_st = base + OFF_A + st * A_BYTES;
+          const uint32_t b_st = base + OFF_B + st * B_BYTES;
+          for (int j = 0; j < GPS; ++j, ++gi) {
+            const int buf = gi % ACC_BUFS;
+            const uint32_t aph = (uint32_t)(gi / ACC_BUFS) & 1u;
+            if (!mbar_wait_bounded(bar_acce + 8 * buf, aph ^ 1u, abort_flag, &g_gemm_status,
+                                   kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // one MMA per 32-wide group: advance 32 bytes inside the swizzled 128-byte rows
+            umma_ss<kKindI8>(tmem_base + (uint32_t)(buf * BN), sw128_kmajor_desc(a_st + 32u * j),
+                             sw128_kmajor_desc(b_st + 32u * j), idesc, 0u);
+            umma_commit(bar_accf + 8 * buf);
+          }
+          if (ok) umma_commit(bar_empty + 8 * st);
         }
-        if (ok) umma_commit(bar_empty + 8 * st);
       }
       // retire every MMA of this CTA before TMEM is released
       umma_commit(bar_drain);
@@ -236,70 +250,76 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int col0 = (warp >> 2) * EPI_COLS;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)col0;
-    float2 acc[EPI_COLS / 2];
-#pragma unroll
-    for (int i = 0; i < EPI_COLS / 2; ++i) acc[i] = make_float2(0.f, 0.f);
     pdl_wait();  // y may be read by a kernel before the previous one
     bool ok = true;
-    for (int gi = 0; gi < G && ok; gi += 2) {
-      const int kb = gi / GPS, j = gi % GPS, st = kb % STAGES;
-      if (j == 0)  // the pair's steps arrive with its stage
-        ok = mbar_wait_bounded(bar_full + 8 * st, (uint32_t)(kb / STAGES) & 1u, abort_flag,
-                               &g_gemm_status, kWaitLimitNs);
-      const int b0 = gi % ACC_BUFS, b1 = (gi + 1) % ACC_BUFS;
-      ok = ok && mbar_wait_bounded(bar_accf + 8 * b1, (uint32_t)((gi + 1) / ACC_BUFS) & 1u,
-                                   abort_flag, &g_gemm_status, kWaitLimitNs);
-      if (!ok) break;
-      tc_fence_after();
-      const float* sa_row = reinterpret_cast<const float*>(gbase + OFF_SA + st * SA_BYTES) + row * 4;
-      const float sa0 = sa_row[j], sa1 = sa_row[j + 1];
-      const float2 s20 = make_float2(sa0, sa0), s21 = make_float2(sa1, sa1);
-      const float4* sw0 =
-          reinterpret_cast<const float4*>(gbase + OFF_SW + st * SW_BYTES) + (j * BN + col0) / 4;
-      const float4* sw1 = sw0 + BN / 4;
-      uint32_t rA[16], rB[16];
+    int kbg0 = 0, gi0 = 0;  // this tile's first k-block and group in the CTA's sequence
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, kbg0 += n_kb, gi0 += G) {
+      const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+      float2 acc[EPI_COLS / 2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // column halves 0-15, 16-31
-        tmem_ld_32x32b_x16(lane_base + (uint32_t)(b0 * BN + 16 * h), rA);
-        tmem_ld_32x32b_x16(lane_base + (uint32_t)(b1 * BN + 16 * h), rB);
-        tmem_wait_ld();
-        if (h == 1) {  // both accumulators fully read: hand the buffers back
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(bar_acce + 8 * b0);
-            mbar_arrive(bar_acce + 8 * b1);
+      for (int i = 0; i < EPI_COLS / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+      for (int g = 0; g < G && ok; g += 2) {
+        const int kbg = kbg0 + g / GPS, j = g % GPS, st = kbg % STAGES;
+        const int gi = gi0 + g;  // G is a multiple of 4, so gi % 4 == g % 4
+        if (j == 0)  // the pair's steps arrive with its stage
+          ok = mbar_wait_bounded(bar_full + 8 * st, (uint32_t)(kbg / STAGES) & 1u, abort_flag,
+                                 &g_gemm_status, kWaitLimitNs);
+        const int b0 = gi % ACC_BUFS, b1 = (gi + 1) % ACC_BUFS;
+        ok = ok && mbar_wait_bounded(bar_accf + 8 * b1, (uint32_t)((gi + 1) / ACC_BUFS) & 1u,
+                                     abort_flag, &g_gemm_status, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        const float* sa_row =
+            reinterpret_cast<const float*>(gbase + OFF_SA + st * SA_BYTES) + row * 4;
+        const float sa0 = sa_row[j], sa1 = sa_row[j + 1];
+        const float2 s20 = make_float2(sa0, sa0), s21 = make_float2(sa1, sa1);
+        const float4* sw0 =
+            reinterpret_cast<const float4*>(gbase + OFF_SW + st * SW_BYTES) + (j * BN + col0) / 4;
+        const float4* sw1 = sw0 + BN / 4;
+        uint32_t rA[16], rB[16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // column halves 0-15, 16-31
+          tmem_ld_32x32b_x16(lane_base + (uint32_t)(b0 * BN + 16 * h), rA);
+          tmem_ld_32x32b_x16(lane_base + (uint32_t)(b1 * BN + 16 * h), rB);
+          tmem_wait_ld();
+          if (h == 1) {  // both accumulators fully read: hand the buffers back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(bar_acce + 8 * b0);
+              mbar_arrive(bar_acce + 8 * b1);
+            }
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const float4 w0 = sw0[4 * h + c4], w1 = sw1[4 * h + c4];
+            float2& a0 = acc[8 * h + 2 * c4];
+            float2& a1 = acc[8 * h + 2 * c4 + 1];
+            a0 = ffma2(fmul2(s20, make_float2(w0.x, w0.y)),
+                       acc_pair<kKindI8>(rA[4 * c4 + 0], rA[4 * c4 + 1]), a0);
+            a1 = ffma2(fmul2(s20, make_float2(w0.z, w0.w)),
+                       acc_pair<kKindI8>(rA[4 * c4 + 2], rA[4 * c4 + 3]), a1);
+            a0 = ffma2(fmul2(s21, make_float2(w1.x, w1.y)),
+                       acc_pair<kKindI8>(rB[4 * c4 + 0], rB[4 * c4 + 1]), a0);
+            a1 = ffma2(fmul2(s21, make_float2(w1.z, w1.w)),
+                       acc_pair<kKindI8>(rB[4 * c4 + 2], rB[4 * c4 + 3]), a1);
           }
         }
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const float4 w0 = sw0[4 * h + c4], w1 = sw1[4 * h + c4];
-          float2& a0 = acc[8 * h + 2 * c4];
-          float2& a1 = acc[8 * h + 2 * c4 + 1];
-          a0 = ffma2(fmul2(s20, make_float2(w0.x, w0.y)),
-                     acc_pair<kKindI8>(rA[4 * c4 + 0], rA[4 * c4 + 1]), a0);
-          a1 = ffma2(fmul2(s20, make_float2(w0.z, w0.w)),
-                     acc_pair<kKindI8>(rA[4 * c4 + 2], rA[4 * c4 + 3]), a1);
-          a0 = ffma2(fmul2(s21, make_float2(w1.x, w1.y)),
-                     acc_pair<kKindI8>(rB[4 * c4 + 0], rB[4 * c4 + 1]), a0);
-          a1 = ffma2(fmul2(s21, make_float2(w1.z, w1.w)),
-                     acc_pair<kKindI8>(rB[4 * c4 + 2], rB[4 * c4 + 3]), a1);
+        if (j + 2 == GPS) {  // this stage's shared-memory steps are no longer needed
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_empty + 8 * st);
         }
       }
-      if (j + 2 == GPS) {  // this stage's shared-memory steps are no longer needed
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_empty + 8 * st);
-      }
-    }
-    const int gm = m0 + row;
-    if (ok && gm < M) {
-      const int64_t j = gm / y_seg_rows;  // loop segment of this row
-      float* yr = y + j * y_stride + (gm - j * y_seg_rows) * (int64_t)N + n0 + col0;
+      const int gm = m0 + row;
+      if (ok && gm < M) {
+        const int64_t jseg = gm / y_seg_rows;  // loop segment of this row
+        float* yr = y + jseg * y_stride + (gm - jseg * y_seg_rows) * (int64_t)N + n0 + col0;
 #pragma unroll
-      for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
-        if (n0 + col0 + 4 * c4 < N)
-          *reinterpret_cast<float4*>(yr + 4 * c4) =
-              make_float4(acc[2 * c4].x, acc[2 * c4].y, acc[2 * c4 + 1].x, acc[2 * c4 + 1].y);
+        for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
+          if (n0 + col0 + 4 * c4 < N)
+            *reinterpret_cast<float4*>(yr + 4 * c4) =
+                make_float4(acc[2 * c4].x, acc[2 * c4].y, acc[2 * c4 + 1].x, acc[2 * c4 + 1].y);
+        }
       }
     }
   }
@@ -371,7 +391,13 @@ cudaError_t launch_impl(const uint8_t* A, const float* sa, const uint8_t* B, con
     if (e != cudaSuccess) return e;
     attr_set_mask |= 1ull << (dev & 63);
   }
-  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  // persistent: one CTA per SM (1 CTA fits per SM), at most one per tile
+  const int64_t n_tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
+  if (n_tiles > INT32_MAX) {
+    if (why) *why = "too many output tiles";
+    return cudaErrorInvalidValue;
+  }
+  dim3 grid((unsigned)std::min<int64_t>(n_tiles, num_sms()));
   return launch_kernel(k, grid, dim3(THREADS), SMEM_BYTES, s, pdl, mA, mB, mSA, mSW, y, (int)M,
                        (int)N, (int)G, y_seg_rows, y_stride);
 }
