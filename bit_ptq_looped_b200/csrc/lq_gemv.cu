@@ -53,9 +53,10 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
   const int W = gridDim.x * kGemvWarps;                 // warps in the grid
   const size_t rowstride = (size_t)K / 2;               // bytes per packed weight row
 
-  uint4 wv[RPW][GPL];
-  float swv[RPW][GPL];
-  auto load_batch = [&](int j0) {  // rows gw + (j0 + r) * W, r < RPW
+  // two register sets of weight rows: batch b + 1 is in flight while batch b is folded
+  uint4 wv[2][RPW][GPL];
+  float swv[2][RPW][GPL];
+  auto load_batch = [&](int buf, int j0) {  // rows gw + (j0 + r) * W, r < RPW
 #pragma unroll
     for (int r = 0; r < RPW; ++r) {
       const int n = gw + (j0 + r) * W;
@@ -63,16 +64,16 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
       for (int gi = 0; gi < GPL; ++gi) {
         const int g = lane + 32 * gi;
         if (n < N && g < G) {
-          wv[r][gi] = __ldg(reinterpret_cast<const uint4*>(w4 + (size_t)n * rowstride) + g);
-          swv[r][gi] = __ldg(sw + (size_t)n * G + g);
+          wv[buf][r][gi] = __ldg(reinterpret_cast<const uint4*>(w4 + (size_t)n * rowstride) + g);
+          swv[buf][r][gi] = __ldg(sw + (size_t)n * G + g);
         } else {
-          wv[r][gi] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-          swv[r][gi] = 0.f;
+          wv[buf][r][gi] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+          swv[buf][r][gi] = 0.f;
         }
       }
     }
   };
-  load_batch(0);
+  load_batch(0, 0);
 
   // ---- the activation: written by the previous kernel of the sequence
   pdl_wait();
@@ -90,8 +91,8 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
   }
   __syncthreads();
 
-  for (int j0 = 0; gw + j0 * W < N; j0 += RPW) {
-    if (j0 > 0) load_batch(j0);
+  // fold batch `buf` (rows gw + (j0 + r) * W) into y
+  auto fold_batch = [&](int buf, int j0) {
     float part[RPW][MB];
 #pragma unroll
     for (int r = 0; r < RPW; ++r)
@@ -104,8 +105,9 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
         uint32_t lo[RPW][4], hi[RPW][4];
 #pragma unroll
         for (int r = 0; r < RPW; ++r) {
-          const uint32_t wu[4] = {wv[r][gi].x ^ 0x88888888u, wv[r][gi].y ^ 0x88888888u,
-                                  wv[r][gi].z ^ 0x88888888u, wv[r][gi].w ^ 0x88888888u};
+          const uint4 w = wv[buf][r][gi];
+          const uint32_t wu[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u,
+                                  w.w ^ 0x88888888u};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             lo[r][i] = wu[i] & 0x0F0F0F0Fu;
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
               d = dp4a_us(hi[r][2], a1.y, d);
               d = dp4a_us(lo[r][3], a1.z, d);
               d = dp4a_us(hi[r][3], a1.w, d);
-              part[r][m] = fmaf(sam * swv[r][gi], (float)(d - corr), part[r][m]);
+              part[r][m] = fmaf(sam * swv[buf][r][gi], (float)(d - corr), part[r][m]);
             }
           }
         }
@@ -153,6 +155,17 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
       for (int m = 0; m < MB; ++m)
         if (lane == ((r * MB + m) & 31) && m < M && n < N) y[(size_t)m * N + n] = part[r][m];
     }
+  };
+
+  // batches alternate between the two register sets (the loop is unrolled by
+  // two so that every register index is static)
+  for (int j0 = 0; gw + j0 * W < N; j0 += 2 * RPW) {
+    const bool more1 = gw + (j0 + RPW) * W < N;
+    if (more1) load_batch(1, j0 + RPW);
+    fold_batch(0, j0);
+    if (!more1) break;
+    if (gw + (j0 + 2 * RPW) * W < N) load_batch(0, j0 + 2 * RPW);
+    fold_batch(1, j0 + RPW);
   }
 }
 
@@ -198,9 +211,10 @@ cudaError_t launch_mb(const int8_t* qa, const int* asum, const float* sa, const 
   const int64_t G = K / kGroup;
   if (G > 128) return launch_cfg<MB, 8, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
   if (G > 64) return launch_cfg<MB, 4, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  // three rows per warp once that still gives every SM one and a half blocks
-  if (N >= (int64_t)num_sms() * kGemvWarps * 3 * 3 / 2)
-    return launch_cfg<MB, 2, 3>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  // up to 4 rows: three weight rows per warp once that still gives every SM
+  // one and a half blocks (16 rows keep one: their partial sums need the registers)
+  if (MB <= 4 && N >= (int64_t)num_sms() * kGemvWarps * 3 * 3 / 2)
+    return launch_cfg<MB, 2, (MB <= 4 ? 3 : 1)>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
   return launch_cfg<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 

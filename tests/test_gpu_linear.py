@@ -87,6 +87,27 @@ def test_loop_linear_decode(M, N, a_bits):
         linear_parity(host(y), x, ol, t, host(q8), host(s), layer.w_flips)
 
 
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_gemv_many_row_batches(M):
+    """N = 3 * 5632 + 8 weight rows: more rows than one resident wave of warps
+    holds, so every warp folds several batches through both register sets of
+    the weight prefetch, and the last batch is ragged."""
+    N = 3 * 5632 + 8
+    wl = synth.Workload(f"decode_M{M}_N{N}", M=M, T=1,
+                        linears=(synth.Linear("dec", 2048, N, 32, 64, 0),), a_bits=8,
+                        outlier_frac=0.02, outlier_mult=20.0, x_dtype="bf16",
+                        description="decode GEMV with several row batches per warp")
+    (mp,) = synth.module_params(wl)
+    (lin,) = wl.linears
+    layer, ol = make_layer(mp, 8)
+    x = synth.loop_input(wl, lin, 0)
+    xd = act_tensor(x, wl.x_dtype)
+    y = lq.lq_loop_linear(xd, layer, 0)
+    q8, _, s = lq.lq_quantize_act(xd, dev(mp.P1), dev(mp.P2), float(mp.las[0]), 8)
+    torch.cuda.synchronize()
+    linear_parity(host(y), x, ol, 0, host(q8), host(s), layer.w_flips)
+
+
 @pytest.mark.parametrize("M", [0, 1, 17, 129, 300])
 def test_loop_linear_ragged_rows(M):
     wl = synth.TINY
