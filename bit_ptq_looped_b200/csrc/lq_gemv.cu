@@ -38,9 +38,10 @@ __device__ __forceinline__ int dp4a_us(uint32_t a_unsigned, uint32_t b_signed, i
 }
 
 // MB: activation rows handled (M <= MB); GPL: group slots per lane (G <= 32 * GPL);
-// RPW: weight rows per warp per batch.
+// RPW: weight rows per warp per batch; kDB: prefetch batch b + 1 while folding b
+// (worth its registers only when a warp has more than one batch).
 // shared layout: act vectors [(m * 2 + h) * G + g] (uint4), then asum[M * G], ssa[M * G].
-template <int MB, int GPL, int RPW>
+template <int MB, int GPL, int RPW, bool kDB>
 __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
     const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
     const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
@@ -53,9 +54,10 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
   const int W = gridDim.x * kGemvWarps;                 // warps in the grid
   const size_t rowstride = (size_t)K / 2;               // bytes per packed weight row
 
-  // two register sets of weight rows: batch b + 1 is in flight while batch b is folded
-  uint4 wv[2][RPW][GPL];
-  float swv[2][RPW][GPL];
+  // register sets of weight rows: with kDB, batch b + 1 is in flight while batch b is folded
+  constexpr int kSets = kDB ? 2 : 1;
+  uint4 wv[kSets][RPW][GPL];
+  float swv[kSets][RPW][GPL];
   auto load_batch = [&](int buf, int j0) {  // rows gw + (j0 + r) * W, r < RPW
 #pragma unroll
     for (int r = 0; r < RPW; ++r) {
@@ -157,26 +159,33 @@ __global__ void __launch_bounds__(kGemvThreads) k_group_gemv(
     }
   };
 
-  // batches alternate between the two register sets (the loop is unrolled by
-  // two so that every register index is static)
-  for (int j0 = 0; gw + j0 * W < N; j0 += 2 * RPW) {
-    const bool more1 = gw + (j0 + RPW) * W < N;
-    if (more1) load_batch(1, j0 + RPW);
-    fold_batch(0, j0);
-    if (!more1) break;
-    if (gw + (j0 + 2 * RPW) * W < N) load_batch(0, j0 + 2 * RPW);
-    fold_batch(1, j0 + RPW);
+  if (kDB) {
+    // batches alternate between the two register sets (the loop is unrolled by
+    // two so that every register index is static)
+    for (int j0 = 0; gw + j0 * W < N; j0 += 2 * RPW) {
+      const bool more1 = gw + (j0 + RPW) * W < N;
+      if (more1) load_batch(kSets - 1, j0 + RPW);
+      fold_batch(0, j0);
+      if (!more1) break;
+      if (gw + (j0 + 2 * RPW) * W < N) load_batch(0, j0 + 2 * RPW);
+      fold_batch(kSets - 1, j0 + RPW);
+    }
+  } else {
+    for (int j0 = 0; gw + j0 * W < N; j0 += RPW) {
+      if (j0 > 0) load_batch(0, j0);
+      fold_batch(0, j0);
+    }
   }
 }
 
 size_t gemv_smem_bytes(int64_t M, int64_t G) { return (size_t)M * G * (32 + 8); }
 
-template <int MB, int GPL, int RPW>
+template <int MB, int GPL, int RPW, bool kDB>
 cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                        const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
                        bool pdl) {
   const size_t smem = gemv_smem_bytes(M, K / kGroup);
-  auto* k = k_group_gemv<MB, GPL, RPW>;
+  auto* k = k_group_gemv<MB, GPL, RPW, kDB>;
   // resident blocks per SM for this instantiation and shared-memory size
   static std::mutex mu;
   static std::unordered_map<size_t, int> per_sm_cache;
@@ -204,18 +213,29 @@ cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const
                        w4, sw, y, (int)M, (int)N, (int)K);
 }
 
+// one batch per warp fits in a resident wave: no prefetch registers needed
+template <int MB, int GPL, int RPW>
+cudaError_t launch_rpw(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
+                       const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                       bool pdl) {
+  const int64_t one_wave_rows = (int64_t)num_sms() * 2 * kGemvWarps * RPW;
+  if (N <= one_wave_rows)
+    return launch_cfg<MB, GPL, RPW, false>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_cfg<MB, GPL, RPW, true>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+}
+
 template <int MB>
 cudaError_t launch_mb(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                       const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
                       bool pdl) {
   const int64_t G = K / kGroup;
-  if (G > 128) return launch_cfg<MB, 8, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  if (G > 64) return launch_cfg<MB, 4, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  if (G > 128) return launch_rpw<MB, 8, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  if (G > 64) return launch_rpw<MB, 4, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
   // up to 4 rows: three weight rows per warp once that still gives every SM
   // one and a half blocks (16 rows keep one: their partial sums need the registers)
   if (MB <= 4 && N >= (int64_t)num_sms() * kGemvWarps * 3 * 3 / 2)
-    return launch_cfg<MB, 2, (MB <= 4 ? 3 : 1)>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  return launch_cfg<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+    return launch_rpw<MB, 2, (MB <= 4 ? 3 : 1)>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_rpw<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
 }  // namespace

@@ -297,10 +297,41 @@ __device__ __forceinline__ void load_row_chunk8(const Tin* __restrict__ x, int64
   d[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// 8 input elements held as raw vectors, so a prefetch does not wait for its data
+template <typename Tin> struct RawChunk;
+template <> struct RawChunk<float> {
+  float4 v0, v1;
+  __device__ __forceinline__ void load(const float* __restrict__ x, int64_t chunk) {
+    const float4* p = reinterpret_cast<const float4*>(x + chunk * 8);
+    v0 = __ldg(p);
+    v1 = __ldg(p + 1);
+  }
+  __device__ __forceinline__ void zero() { v0 = v1 = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void store(float* dst) const {
+    reinterpret_cast<float4*>(dst)[0] = v0;
+    reinterpret_cast<float4*>(dst)[1] = v1;
+  }
+};
+template <> struct RawChunk<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* __restrict__ x, int64_t chunk) {
+    v = __ldg(reinterpret_cast<const uint4*>(x + chunk * 8));
+  }
+  __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void store(float* dst) const {
+    reinterpret_cast<float4*>(dst)[0] =
+        make_float4(bf16_bits_to_f32(v.x & 0xFFFFu), bf16_bits_to_f32(v.x >> 16),
+                    bf16_bits_to_f32(v.y & 0xFFFFu), bf16_bits_to_f32(v.y >> 16));
+    reinterpret_cast<float4*>(dst)[1] =
+        make_float4(bf16_bits_to_f32(v.z & 0xFFFFu), bf16_bits_to_f32(v.z >> 16),
+                    bf16_bits_to_f32(v.w & 0xFFFFu), bf16_bits_to_f32(v.w >> 16));
+  }
+};
+
 constexpr int kRotTM = 2, kRotTN = 4;  // warp task: 16 x 32 outputs
 
 template <typename Tin, bool kStoreF32>
-__global__ void __launch_bounds__(kThreads) k_rotate_quant(
+__global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
     const Tin* __restrict__ x, int64_t M, int K, const float* __restrict__ P1, int a,
     const float* __restrict__ P2, int b, int R, const LoopSegs segs, int qmax,
     int8_t* __restrict__ codes8,
@@ -327,27 +358,28 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
   const int row_chunks = K >> 3;
   const FastDiv fd_rowc((uint32_t)row_chunks), fd_b((uint32_t)b), fd_a((uint32_t)a);
 
-  // ---- prologue: the first tile's input and the factors are loaded with all
-  // loads of a thread in flight at once (one memory round trip, not one per
-  // element: for a few rows this latency is most of the kernel's time)
+  // ---- input tiles are prefetched into registers as raw vectors: the first
+  // one here, together with the factors (one memory round trip, not one per
+  // element: for a few rows this latency is most of the kernel's time), and
+  // each next one at the start of the previous tile's MMA stages
   constexpr int kXU = 2, kFU = 24;
-  const int64_t m_first = (int64_t)blockIdx.x * R;
-  const bool x_pre = x_early && R * row_chunks <= kXU * kThreads;
-  float xr[kXU][8];
-  if (x_pre) {
+  // (without x_early the kernel has already waited for its predecessor above)
+  const bool x_pre = R * row_chunks <= kXU * kThreads;
+  RawChunk<Tin> xr[kXU];
+  auto prefetch_tile = [&](int64_t m0p) {
 #pragma unroll
     for (int u = 0; u < kXU; ++u) {
       const int ch = u * kThreads + tid;
       const int r = (int)fd_rowc.div((uint32_t)ch);
-      if (ch < R * row_chunks && m_first + r < M) {
-        const int64_t gr = m_first + r, j = gr / segs.seg_rows;
-        load8(x + j * segs.x_stride + (gr - j * segs.seg_rows) * K, ch - r * row_chunks, xr[u]);
+      if (ch < R * row_chunks && m0p + r < M) {
+        const int64_t gr = m0p + r, j = gr / segs.seg_rows;
+        xr[u].load(x + j * segs.x_stride + (gr - j * segs.seg_rows) * K, ch - r * row_chunks);
       } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xr[u][e] = 0.f;
+        xr[u].zero();
       }
     }
-  }
+  };
+  if (x_pre) prefetch_tile((int64_t)blockIdx.x * R);
   {
     const int n2 = b * b, nf = n2 + a * a;
     for (int base = 0; base < nf; base += kFU * kThreads) {
@@ -382,7 +414,6 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
   const FastDiv fd_s1ctq((uint32_t)s1_ctq), fd_s2tok((uint32_t)(s2_rt * s1_ctq));
 
   int par = 0;
-  bool first = true;
   for (int64_t m0 = (int64_t)blockIdx.x * R; m0 < M; m0 += (int64_t)gridDim.x * R, par ^= 1) {
     const int rows = (M - m0 < (int64_t)R) ? (int)(M - m0) : R;
     if (tid < rows) {
@@ -395,16 +426,14 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
       row_c[par][tid] = cj;
     }
     __syncthreads();  // previous Z consumed; factors and row offsets staged
-    if (first && x_pre) {  // the prologue's registers (zeros past the last row)
+    if (x_pre) {  // the prefetched registers (zeros past the last row)
 #pragma unroll
       for (int u = 0; u < kXU; ++u) {
         const int ch = u * kThreads + tid;
         if (ch < R * row_chunks) {
           const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
           const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
-          float4* dst = reinterpret_cast<float4*>(X + (size_t)(r * a + i) * L.ldb + q);
-          dst[0] = make_float4(xr[u][0], xr[u][1], xr[u][2], xr[u][3]);
-          dst[1] = make_float4(xr[u][4], xr[u][5], xr[u][6], xr[u][7]);
+          xr[u].store(X + (size_t)(r * a + i) * L.ldb + q);
         }
       }
     } else {
@@ -420,8 +449,9 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant(
         }
       }
     }
-    first = false;
     __syncthreads();
+    // the next tile's input is in flight during this tile's MMA stages
+    if (x_pre && m0 + (int64_t)gridDim.x * R < M) prefetch_tile(m0 + (int64_t)gridDim.x * R);
     // ---- stage 1: Y[(r,i), j] = sum_q X[(r,i), q] P2[q, j]  -> YT[r][j][i]
     for (int task = warp; task < s1_tasks; task += kWarps) {
       const int rt = (int)fd_s1ctq.div((uint32_t)task), cq = task - rt * s1_ctq;
