@@ -528,6 +528,167 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
   }
 }
 
+// ---------------------------------------------------------------------------
+// fused rotation + quantization for a few token rows (decode)
+//
+// With only a handful of rows the row-tile kernel above leaves most SMs idle
+// and each block's time is mostly load and MMA latency.  Here block (row m,
+// slice s) computes the 32 columns J = [32s, 32s + 32) of Z = P1^T X P2 for
+// one row: Y_J = X P2[:, J] (a x 32, b-long dots), then Z_J = P1^T Y_J (a-long
+// dots), both on the FP64 tensor-core MMA like the row-tile kernel, rounded
+// once to float32.  When b is a multiple of 32, row i of Z_J is exactly
+// quantization group i * b/32 + s, so each block quantizes whole groups.
+// Shared-memory operands, row pitches padded by 4 elements:
+//   X[i][q] f32 (a x b), P2T[j][q] = P2[q][32s + j] (32 x b), P1T[i][p] = P1[p][i]
+//   (a x a), YT[j][p] = Y_J[p][j] (32 x a), Z[i][j] f32 (a x 32).
+// ---------------------------------------------------------------------------
+constexpr int kSmallMaxA = 64, kSmallMaxB = 128;
+constexpr int64_t kSmallRotMaxRows = 16;  // up to the decode GEMV's row limit
+
+struct SmallRotLayout {
+  int ldx, ldp2, ldp1, ldy, ldz;
+  size_t off_p2t, off_p1t, off_yt, off_x, off_z, bytes;  // byte offsets
+};
+
+__host__ __device__ inline SmallRotLayout small_rot_layout(int a, int b) {
+  SmallRotLayout L;
+  L.ldx = b + 4;
+  L.ldp2 = b + 4;
+  L.ldp1 = a + 4;
+  L.ldy = a + 4;
+  L.ldz = 32 + 4;
+  L.off_p2t = 0;
+  L.off_p1t = L.off_p2t + 8 * (size_t)32 * L.ldp2;
+  L.off_yt = L.off_p1t + 8 * (size_t)a * L.ldp1;
+  L.off_x = L.off_yt + 8 * (size_t)32 * L.ldy;
+  L.off_z = L.off_x + 4 * (size_t)a * L.ldx;
+  L.bytes = L.off_z + 4 * (size_t)a * L.ldz;
+  return L;
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
+    const Tin* __restrict__ x, int K, const float* __restrict__ P1, int a,
+    const float* __restrict__ P2, int b, const LoopSegs segs, int qmax,
+    int8_t* __restrict__ codes8, int opf, uint8_t* __restrict__ codes4,
+    float* __restrict__ scales, int* __restrict__ asum, int x_early) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  if (!x_early) pdl_wait();
+  const int tid = threadIdx.x, warp = tid >> 5;
+  constexpr int kWarps = kThreads / 32;
+  const int S = b >> 5;
+  const int m = blockIdx.x / S, sl = blockIdx.x - m * S;
+  const SmallRotLayout L = small_rot_layout(a, b);
+  double* P2T = reinterpret_cast<double*>(smem_raw + L.off_p2t);
+  double* P1T = reinterpret_cast<double*>(smem_raw + L.off_p1t);
+  double* YT = reinterpret_cast<double*>(smem_raw + L.off_yt);
+  float* Xs = reinterpret_cast<float*>(smem_raw + L.off_x);
+  float* Zs = reinterpret_cast<float*>(smem_raw + L.off_z);
+  const FastDiv fd_b((uint32_t)b), fd_a((uint32_t)a);
+
+  // ---- loads, all of a thread's in flight together
+  const int64_t jseg = (int64_t)m / segs.seg_rows;
+  const Tin* xrow = x + jseg * segs.x_stride + ((int64_t)m - jseg * segs.seg_rows) * K;
+  float c = segs.c[0];  // static indices keep the parameter block out of local memory
+#pragma unroll
+  for (int u = 1; u < kMaxLoopsPerLaunch; ++u)
+    if (jseg == u) c = segs.c[u];
+  {
+    constexpr int kP2U = kSmallMaxB * 32 / kThreads, kP1U = kSmallMaxA * kSmallMaxA / kThreads;
+    constexpr int kXU = kSmallMaxA * kSmallMaxB / 8 / kThreads;
+    const int n2 = b * 32, n1 = a * a, nx = K >> 3;  // P2 slice, P1, input chunks of 8
+    float p2v[kP2U], p1v[kP1U];
+    RawChunk<Tin> xv[kXU];
+#pragma unroll
+    for (int u = 0; u < kXU; ++u)
+      if (u * kThreads + tid < nx) xv[u].load(xrow, u * kThreads + tid);
+#pragma unroll
+    for (int u = 0; u < kP2U; ++u) {  // element (q, j) = (e / 32, e % 32) of the slice
+      const int e = u * kThreads + tid;
+      p2v[u] = e < n2 ? __ldg(P2 + (size_t)(e >> 5) * b + 32 * sl + (e & 31)) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kP1U; ++u) {
+      const int e = u * kThreads + tid;
+      p1v[u] = e < n1 ? __ldg(P1 + e) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kXU; ++u) {
+      const int ch = u * kThreads + tid;
+      if (ch < nx) {
+        const int k8 = ch * 8, i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
+        xv[u].store(Xs + (size_t)i * L.ldx + q);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kP2U; ++u) {
+      const int e = u * kThreads + tid;
+      if (e < n2) P2T[(size_t)(e & 31) * L.ldp2 + (e >> 5)] = (double)p2v[u];
+    }
+#pragma unroll
+    for (int u = 0; u < kP1U; ++u) {
+      const int e = u * kThreads + tid;
+      if (e < n1) {
+        const int pp = (int)fd_a.div((uint32_t)e), i = e - pp * a;
+        P1T[(size_t)i * L.ldp1 + pp] = (double)p1v[u];
+      }
+    }
+  }
+  __syncthreads();
+
+  // warp tasks of 8 x 16 outputs: (a / 8) row tiles x 2 column pairs
+  const int n_tasks = (a >> 3) * 2;
+  // ---- Y_J[p][j] = sum_q X[p][q] P2[q][32 s + j]  -> YT[j][p]
+  for (int task = warp; task < n_tasks; task += kWarps) {
+    warp_mma_task<1, 2>(Xs, L.ldx, P2T, L.ldp2, b, (task >> 1) * 8, (task & 1) * 2, 4,
+                        [&](int pp, int j, double v0, double v1) {
+                          YT[(size_t)j * L.ldy + pp] = v0;
+                          YT[(size_t)(j + 1) * L.ldy + pp] = v1;
+                        });
+  }
+  __syncthreads();
+  // ---- Z_J[i][j] = sum_p P1[p][i] Y_J[p][j], rounded once to float32
+  for (int task = warp; task < n_tasks; task += kWarps) {
+    warp_mma_task<1, 2>(P1T, L.ldp1, YT, L.ldy, a, (task >> 1) * 8, (task & 1) * 2, 4,
+                        [&](int i, int j, double v0, double v1) {
+                          *reinterpret_cast<float2*>(Zs + (size_t)i * L.ldz + j) =
+                              make_float2(__double2float_rn(v0), __double2float_rn(v1));
+                        });
+  }
+  __syncthreads();
+  if (x_early) pdl_wait();  // the previous kernel may still read the output buffers
+
+  // ---- quantize: thread t takes chunk t % 4 (8 values) of group row t / 4
+  const int G = K / kGroup;
+  for (int base = 0; base < a * 4; base += kThreads) {
+    if (base + (tid & ~31) >= a * 4) break;  // whole warp past the last group
+    const int t = base + tid;
+    const bool valid = t < a * 4;
+    const int i = t >> 2, cq = t & 3;
+    float v[8];
+    if (valid) {
+      const float4* src = reinterpret_cast<const float4*>(Zs + (size_t)i * L.ldz + 8 * cq);
+      const float4 u0 = src[0], u1 = src[1];
+      v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+      v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    }
+    uint32_t q[8];
+    const float st = quant_group8(v, c, qmax, q);
+    // chunk of element i * b + 32 s + 8 cq of row m
+    const int64_t chunk = ((int64_t)m * K + (int64_t)i * b + 32 * sl + 8 * cq) >> 3;
+    if (opf == kOpGemvAct) {
+      const int gs = group_code_sum(q);
+      if (valid) store_codes<true>(q, st, chunk, codes8, opf, codes4, scales, G, gs, asum);
+    } else if (valid) {
+      store_codes<false>(q, st, chunk, codes8, opf, codes4, scales);
+    }
+  }
+}
+
 __global__ void k_codes4_to_operand(const uint8_t* __restrict__ codes4, int64_t n_words, int opf,
                                     uint8_t* __restrict__ out) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -614,6 +775,23 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
     return launch_kernel(gv ? k_quant_only<float, true> : k_quant_only<float, false>, dim3(grid),
                          dim3(kThreads), 0, s, pdl, (const float*)x, n_chunks, c, qmax, codes8,
                          opf, codes4, scales, G, asum, xe);
+  }
+  if (M <= kSmallRotMaxRows && b % 32 == 0 && a <= kSmallMaxA && b <= kSmallMaxB) {
+    // a few rows: one block per (row, 32-column slice) on the FP64 FMA units
+    const size_t ssm = small_rot_layout(a, b).bytes;
+    const int grid = (int)(M * (b / 32));
+    cudaError_t e;
+    if (x_dtype == LQ_BF16) {
+      auto* k = k_rotate_quant_small<__nv_bfloat16>;
+      if ((e = set_smem(k, ssm)) != cudaSuccess) return e;
+      return launch_kernel(k, dim3(grid), dim3(kThreads), ssm, s, pdl, (const __nv_bfloat16*)x,
+                           (int)K, P1, a, P2, b, segs, qmax, codes8, opf, codes4, scales, asum,
+                           xe);
+    }
+    auto* k = k_rotate_quant_small<float>;
+    if ((e = set_smem(k, ssm)) != cudaSuccess) return e;
+    return launch_kernel(k, dim3(grid), dim3(kThreads), ssm, s, pdl, (const float*)x, (int)K,
+                         P1, a, P2, b, segs, qmax, codes8, opf, codes4, scales, asum, xe);
   }
   int R = 0;
   size_t smem = rotate_smem_bytes(a, b, &R);

@@ -88,6 +88,36 @@ def test_fused_rotate_quantize(wl, bits):
             assert len(flips) == 0
 
 
+def _orthogonal(n, seed):
+    q, _ = np.linalg.qr(np.random.default_rng(seed).standard_normal((n, n)))
+    return q.astype(np.float32)
+
+
+@pytest.mark.parametrize("M", [1, 3, 16, 17])
+@pytest.mark.parametrize("ab", [(32, 64), (64, 64), (16, 128), (64, 88), (16, 16)])
+@pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
+def test_fused_rotate_quantize_few_rows(M, ab, x_dtype):
+    """Up to 16 rows with b % 32 == 0 take the one-block-per-(row, 32 columns)
+    kernel; other factor sizes and 17 rows take the row-tile kernel.  Both
+    must give the oracle's codes (only near-tie differences allowed)."""
+    a, b = ab
+    K = a * b
+    x = _outlier_matrix(M, K, seed=M * 131 + K)
+    if x_dtype == "bf16":
+        x = synth.round_bf16(x)
+    P1, P2 = _orthogonal(a, a + 1), _orthogonal(b, b + 2)
+    for bits in (4, 8):
+        q8, q4, s = lq.lq_quantize_act(act_tensor(x, x_dtype), dev(P1), dev(P2), 0.83, bits,
+                                       want_codes4=(bits == 4))
+        torch.cuda.synchronize()
+        xt64 = O.kron_rotate_f64(x, P1, P2)
+        q_or, s_or = O.quantize_groups(xt64.astype(np.float32), 0.83, bits)
+        flips = check_codes_near_tie(host(q8), host(s), q_or, s_or, xt64)
+        assert len(flips) == 0
+        if bits == 4:
+            np.testing.assert_array_equal(O.unpack_int4(host(q4)), host(q8))
+
+
 def test_fused_rotation_identity_factors_reduce_to_plain_rtn():
     M, K = 100, 2048
     x = _outlier_matrix(M, K, seed=3)
