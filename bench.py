@@ -345,6 +345,58 @@ def aux_hbm_kernels(lq, torch, dev, stream, timed, peaks):
     return out
 
 
+def aux_schedules(lq, torch, dev, stream, timed, wl, params, layers, x_dev, ops_step):
+    """The same step under other schedules of the loop driver: loop by loop
+    (workspace for one loop), and SLT serving with every module selected (its
+    own transform and weight at every loop, so no loop shares a launch)."""
+    out = {}
+    M, T, L = wl.M, wl.T, len(wl.linears)
+    y = torch.empty(T * M * sum(lin.N for lin in wl.linears), dtype=torch.float32, device=dev)
+    n = 50
+
+    ws1 = lq.workspace(layers, M, dev)
+    run = lambda: lq.lq_loop_stack(x_dev, layers, T, lq.LQ_OPEN, M=M, y=y, ws=ws1,
+                                   stream=stream)
+    for _ in range(3):
+        run()
+    ms = timed(n, run) / n
+    out["loop_by_loop"] = {"ms_per_step": ms, "TOPS": ops_step / (ms * 1e-3) / 1e12,
+                           "launches_per_step": 2 * T * L}
+
+    rng = np.random.default_rng(17)
+    own, keep = [], []
+    for t in range(T):
+        row = []
+        for mp in params:
+            a, b = mp.P1.shape[0], mp.P2.shape[0]
+            P1 = np.linalg.qr(rng.standard_normal((a, a)))[0].astype(np.float32)
+            P2 = np.linalg.qr(rng.standard_normal((b, b)))[0].astype(np.float32)
+            Q1 = lq.lq_inverse_transpose(P1).to(dev)
+            Q2 = lq.lq_inverse_transpose(P2).to(dev)
+            Wf = lq.lq_fold_weights(torch.from_numpy(mp.W).to(dev), Q1, Q2)
+            wq = lq.lq_pack_weights(Wf)
+            del Wf
+            row.append(lq.lq_layer_create(wq, torch.from_numpy(P1).to(dev),
+                                          torch.from_numpy(P2).to(dev), mp.las, wl.a_bits))
+            keep.append(wq)
+        own.append(row)
+    ws2 = lq.workspace(layers, M, dev, T=T)
+    run = lambda: lq.lq_loop_stack_slt(x_dev, own, lq.LQ_OPEN, M=M, y=y, ws=ws2, stream=stream)
+    for _ in range(3):
+        run()
+    ms = timed(n, run) / n
+    shared_bytes = sum(l.wq.info()["device_bytes"] for l in layers)
+    out["slt_all_selected"] = {"ms_per_step": ms, "TOPS": ops_step / (ms * 1e-3) / 1e12,
+                               "resident_weight_bytes": T * shared_bytes,
+                               "shared_weight_bytes": shared_bytes}
+    for row in own:
+        for l in row:
+            l.free()
+    for wq in keep:
+        wq.free()
+    return out
+
+
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
@@ -495,6 +547,8 @@ def run_lq(args, rank, world, local_rank):
     aux = None
     if not args.no_aux:
         aux = aux_hbm_kernels(lq, torch, dev, stream, timed, load_peaks())
+        aux.update(aux_schedules(lq, torch, dev, stream, timed, wl, params, layers, x_dev,
+                                 ops_step))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

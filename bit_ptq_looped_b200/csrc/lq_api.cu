@@ -654,33 +654,41 @@ lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_l
   return enqueue_linear(d_x, x_dtype, M, layer, t, d_y, d_ws, (cudaStream_t)stream);
 }
 
+// The T x L schedule over a table of handles: step (t, l) applies tl[t * L + l].
 static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
-                               const lq_layer* const* layers, int32_t L, int32_t T, int32_t mode,
-                               float* d_y, void* d_ws, int64_t ws_bytes, cudaStream_t s) {
+                               const std::vector<const lq_layer*>& tl, int32_t L, int32_t T,
+                               int32_t mode, float* d_y, void* d_ws, int64_t ws_bytes,
+                               cudaStream_t s) {
   const size_t esz = x_dtype == LQ_BF16 ? 2 : 4;
+  auto at = [&](int t, int l) { return tl[(size_t)t * L + l]; };
   if (mode == LQ_OPEN) {
     // step (t, l) reads x at element offset M * (t * sum_K + sum_{l' < l} K_l') and
     // writes y at M * (t * sum_N + sum_{l' < l} N_l'); loops of a layer are
-    // independent, so up to loops_per_launch of them share one launch
+    // independent, so consecutive loops that use the same handle share launches
     int64_t sum_k = 0, sum_n = 0;
     for (int l = 0; l < L; ++l) {
-      sum_k += layers[l]->wq->K;
-      sum_n += layers[l]->wq->N;
+      sum_k += at(0, l)->wq->K;
+      sum_n += at(0, l)->wq->N;
     }
     int nb_all = kMaxLoopsPerLaunch;
-    for (int l = 0; l < L; ++l) nb_all = std::min(nb_all, loops_per_launch(layers[l], M, T, ws_bytes));
+    for (const lq_layer* ly : tl) nb_all = std::min(nb_all, loops_per_launch(ly, M, T, ws_bytes));
     bool first = true;
     for (int t = 0; t < T; t += nb_all) {
       const int nb = std::min(nb_all, T - t);
       int64_t k_before = 0, n_before = 0;
       for (int l = 0; l < L; ++l) {
-        const lq_layer* ly = layers[l];
-        const char* xin = (const char*)d_x + (size_t)(M * (t * sum_k + k_before)) * esz;
-        float* yout = d_y + M * (t * sum_n + n_before);
-        lq_status st = enqueue_linear(xin, x_dtype, M, ly, t, yout, d_ws, s, !first, true, nb,
-                                      M * sum_k, M * sum_n);
-        if (st != LQ_OK) return st;
-        first = false;
+        const lq_layer* ly = at(t, l);
+        bool same = true;  // one handle for every loop of the batch
+        for (int j = 1; j < nb; ++j) same = same && at(t + j, l) == ly;
+        for (int j = 0; j < nb; j += same ? nb : 1) {
+          const int w = same ? nb : 1;
+          const char* xin = (const char*)d_x + (size_t)(M * ((t + j) * sum_k + k_before)) * esz;
+          float* yout = d_y + M * ((t + j) * sum_n + n_before);
+          lq_status st = enqueue_linear(xin, x_dtype, M, at(t + j, l), t + j, yout, d_ws, s,
+                                        !first, true, w, M * sum_k, M * sum_n);
+          if (st != LQ_OK) return st;
+          first = false;
+        }
         k_before += ly->wq->K;
         n_before += ly->wq->N;
       }
@@ -691,7 +699,7 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
   const float* prev_y = nullptr;
   for (int t = 0; t < T; ++t) {
     for (int l = 0; l < L; ++l) {
-      const lq_layer* ly = layers[l];
+      const lq_layer* ly = at(t, l);
       const void* xin = prev_y ? (const void*)prev_y : d_x;
       const int32_t dt = prev_y ? LQ_F32 : x_dtype;
       // every linear after the first overlaps its predecessor; its input is
@@ -706,27 +714,39 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
   return LQ_OK;
 }
 
-lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
-                        const lq_layer* const* layers, int32_t L, int32_t T, int32_t mode,
-                        float* d_y, void* d_ws, int64_t ws_bytes, void* stream) {
-  if (!layers || L <= 0 || T <= 0) {
-    set_error("need at least one layer and one loop");
-    return LQ_ERR_ARG;
-  }
+// Checks, graph cache and launch of the schedule over a (t, l) table of handles.
+static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
+                                 const std::vector<const lq_layer*>& tl, int32_t L, int32_t T,
+                                 int32_t mode, float* d_y, void* d_ws, int64_t ws_bytes,
+                                 void* stream) {
   if (mode != LQ_OPEN && mode != LQ_CHAIN) {
     set_error("unknown mode %d", mode);
     return LQ_ERR_ARG;
   }
   lq_status st;
-  for (int l = 0; l < L; ++l) {
-    if ((st = check_layer_call(layers[l], M, x_dtype)) != LQ_OK) return st;
-    if (layers[l]->T < T) {
-      set_error("layer %d has %d LAS clips but T=%d", l, layers[l]->T, T);
-      return LQ_ERR_SHAPE;
+  int64_t need = 0;
+  for (int t = 0; t < T; ++t) {
+    for (int l = 0; l < L; ++l) {
+      const lq_layer* ly = tl[(size_t)t * L + l];
+      if ((st = check_layer_call(ly, M, x_dtype)) != LQ_OK) return st;
+      if (ly->T <= t) {
+        set_error("layer (t=%d, l=%d) has %d LAS clips", t, l, ly->T);
+        return LQ_ERR_SHAPE;
+      }
+      const lq_layer* l0 = tl[l];
+      if (ly->wq->K != l0->wq->K || ly->wq->N != l0->wq->N) {
+        set_error("layer (t=%d, l=%d) is %lldx%lld, loop 0 has %lldx%lld", t, l,
+                  (long long)ly->wq->N, (long long)ly->wq->K, (long long)l0->wq->N,
+                  (long long)l0->wq->K);
+        return LQ_ERR_SHAPE;
+      }
+      need = std::max(need, ws_bytes_for(M, ly->wq->K));
     }
-    if (mode == LQ_CHAIN) {
-      const int64_t next_k = layers[(l + 1) % L]->wq->K;
-      if (layers[l]->wq->N != next_k) {
+  }
+  if (mode == LQ_CHAIN) {
+    for (int l = 0; l < L; ++l) {
+      const int64_t next_k = tl[(l + 1) % L]->wq->K;
+      if (tl[l]->wq->N != next_k) {
         set_error("chain mode needs N_%d == K_%d", l, (l + 1) % L);
         return LQ_ERR_SHAPE;
       }
@@ -741,7 +761,7 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
     set_error("x and y must be 16-byte aligned and the workspace 256-byte aligned");
     return LQ_ERR_ALIGN;
   }
-  if (ws_bytes < lq_workspace_bytes(layers, L, M)) {
+  if (ws_bytes < need) {
     set_error("workspace too small");
     return LQ_ERR_WORKSPACE;
   }
@@ -750,19 +770,14 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   cudaError_t e = cudaStreamIsCapturing(s, &cap);
   if (e != cudaSuccess) return cuda_error(e, "stream query");
-  bool probing;
-  {
-    std::lock_guard<std::mutex> lk(g_probe.mu);
-    probing = g_probe.on;
-  }
-  if (cap != cudaStreamCaptureStatusNone || probing)
-    return enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, ws_bytes, s);
+  if (cap != cudaStreamCaptureStatusNone || probe_on())
+    return enqueue_stack(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, s);
 
   GraphKey key;
   key.x = d_x;
   key.dtype = x_dtype;
   key.M = M;
-  for (int l = 0; l < L; ++l) key.layer_ids.push_back(layers[l]->id);
+  for (const lq_layer* ly : tl) key.layer_ids.push_back(ly->id);
   key.T = T;
   key.mode = mode;
   key.y = d_y;
@@ -784,7 +799,7 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
     }
     if ((e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal)) != cudaSuccess)
       return cuda_error(e, "begin capture");
-    st = enqueue_stack(d_x, x_dtype, M, layers, L, T, mode, d_y, d_ws, ws_bytes, cs);
+    st = enqueue_stack(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, cs);
     cudaGraph_t g = nullptr;
     e = cudaStreamEndCapture(cs, &g);
     if (st != LQ_OK) {
@@ -801,6 +816,36 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
   e = cudaGraphLaunch(it->second, s);
   if (e != cudaSuccess) return cuda_error(e, "graph launch");
   return LQ_OK;
+}
+
+lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
+                        const lq_layer* const* layers, int32_t L, int32_t T, int32_t mode,
+                        float* d_y, void* d_ws, int64_t ws_bytes, void* stream) {
+  if (!layers || L <= 0 || T <= 0) {
+    set_error("need at least one layer and one loop");
+    return LQ_ERR_ARG;
+  }
+  for (int l = 0; l < L; ++l) {
+    if (layers[l] && layers[l]->T < T) {
+      set_error("layer %d has %d LAS clips but T=%d", l, layers[l]->T, T);
+      return LQ_ERR_SHAPE;
+    }
+  }
+  std::vector<const lq_layer*> tl((size_t)T * L);
+  for (int t = 0; t < T; ++t)
+    for (int l = 0; l < L; ++l) tl[(size_t)t * L + l] = layers[l];
+  return loop_stack_impl(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, stream);
+}
+
+lq_status lq_loop_stack_slt(const void* d_x, int32_t x_dtype, int64_t M,
+                            const lq_layer* const* layers_tl, int32_t L, int32_t T, int32_t mode,
+                            float* d_y, void* d_ws, int64_t ws_bytes, void* stream) {
+  if (!layers_tl || L <= 0 || T <= 0) {
+    set_error("need at least one layer and one loop");
+    return LQ_ERR_ARG;
+  }
+  std::vector<const lq_layer*> tl(layers_tl, layers_tl + (size_t)T * L);
+  return loop_stack_impl(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, stream);
 }
 
 lq_status lq_probe_enable(int32_t on) {

@@ -48,6 +48,7 @@ SIGNATURES = {
     "lq_stack_workspace_bytes": (_i64, [_pp, _i32, _i64, _i32]),
     "lq_loop_linear": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
+    "lq_loop_stack_slt": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
     "lq_check_device": (_i32, [_vp]),
     "lq_selftest_bounded_wait": (_i32, [_i64, _vp]),
     "lq_loop_linear_noalloc": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp]),
@@ -310,6 +311,30 @@ def lq_loop_stack(x: torch.Tensor, layers: Sequence[Layer], T: int, mode: int = 
     st = lib().lq_loop_stack(_dev(x, "x"), dt, M, p, len(layers), T, mode, _dev(y, "y"),
                              _dev(ws, "ws"), ws.numel(), _stream(stream))
     _check(st, "lq_loop_stack")
+    return y
+
+
+def lq_loop_stack_slt(x: torch.Tensor, layers_tl: Sequence[Sequence[Layer]], mode: int = LQ_OPEN,
+                      *, M: int, y: Optional[torch.Tensor] = None,
+                      ws: Optional[torch.Tensor] = None, x_dtype: Optional[int] = None,
+                      stream=None) -> torch.Tensor:
+    """layers_tl[t][l]: the handle of module l at loop t (a shared module repeats
+    its handle).  x and y as in lq_loop_stack."""
+    T, L = len(layers_tl), len(layers_tl[0])
+    flat = [layers_tl[t][l] for t in range(T) for l in range(L)]
+    if any(len(row) != L for row in layers_tl):
+        raise ValueError("every loop needs L handles")
+    if y is None:
+        y = torch.empty(T * M * sum(l.N for l in layers_tl[0]), dtype=torch.float32,
+                        device=x.device)
+    if ws is None:
+        uniq = list({id(h): h for h in flat}.values())
+        ws = workspace(uniq, M, x.device, T=T if mode == LQ_OPEN else None)
+    p, keep = _layer_array(flat)
+    dt = _dtype_code(x) if x_dtype is None else x_dtype
+    st = lib().lq_loop_stack_slt(_dev(x, "x"), dt, M, p, L, T, mode, _dev(y, "y"),
+                                 _dev(ws, "ws"), ws.numel(), _stream(stream))
+    _check(st, "lq_loop_stack_slt")
     return y
 
 

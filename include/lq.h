@@ -214,6 +214,29 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
                         float* d_y, void* d_ws, int64_t ws_bytes, void* stream);
 
 /*
+ * lq_loop_stack_slt -- the loop schedule with loop-dependent transforms and
+ * weights for the modules that selective loop-specific transforms (SLT)
+ * picked ("paper_specification.yaml" of the LoopQ reproduction: slt, Section
+ * 4.2 and Eqs. (5)-(6): selected transform-weight groups receive
+ * loop-dependent transforms and weights; Appendix B.1 Table 4 and the
+ * slt_budget, 4 groups on Ouro-1.4B).  The selection itself is calibration
+ * and not part of this library; this call serves a selection.
+ *   layers_tl  T*L handles ordered (t, l): step (t, l) applies
+ *              layers_tl[t*L + l] with that handle's LAS clip c_t.  A module
+ *              that SLT did not select repeats its shared handle in every
+ *              loop; a selected module has one handle per loop (its own P_t,
+ *              folded W_t and clips).  Every handle of module l must have the
+ *              K and N of layers_tl[l], and at least t + 1 clips.
+ * Everything else (modes, input and output layout, workspace, graph reuse,
+ * programmatic launch, errors) as lq_loop_stack, which is this call with
+ * layers_tl[t*L + l] = layers[l].  In open mode, consecutive loops of a module
+ * share launches only where they share a handle.
+ */
+lq_status lq_loop_stack_slt(const void* d_x, int32_t x_dtype, int64_t M,
+                            const lq_layer* const* layers_tl, int32_t L, int32_t T, int32_t mode,
+                            float* d_y, void* d_ws, int64_t ws_bytes, void* stream);
+
+/*
  * lq_loop_linear_noalloc -- lq_loop_linear for callers that cannot allocate
  * device memory, so cannot provide its workspace: for instance the enqueue
  * hook of another runtime that hands over only input and output buffers, a

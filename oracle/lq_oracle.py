@@ -256,3 +256,27 @@ def loop_stack_chain(x0: np.ndarray, layers, T: int):
             cur = y.astype(np.float32)
         ys.append(row)
     return ys
+
+
+def loop_stack_slt_open(xs, layers_tl, T: int):
+    """SLT serving ("paper_specification.yaml" of the LoopQ reproduction: slt,
+    Section 4.2, Eqs. (5)-(6)): the modules SLT selected carry a loop-dependent
+    transform and weight, so step (t, l) applies its own layer layers_tl[t][l];
+    the others repeat their shared layer.  Open mode: input xs[t][l]."""
+    return [[loop_linear(xs[t][l], layers_tl[t][l], t) for l in range(len(layers_tl[t]))]
+            for t in range(T)]
+
+
+def loop_stack_slt_chain(x0: np.ndarray, layers_tl, T: int):
+    """SLT serving in chain mode: y_{t,l} (carried in float32) feeds step (t, l+1)."""
+    ys = []
+    cur = np.asarray(x0, np.float32)
+    for t in range(T):
+        row = []
+        for layer in layers_tl[t]:
+            y = loop_linear(cur, layer, t)
+            row.append(y)
+            cur = y.astype(np.float32)
+        ys.append(row)
+    return ys
+

@@ -1,5 +1,7 @@
 """GPU parity of the quantized looped linear (lq_loop_linear, lq_loop_stack):
 tensor-core GEMM for prefill-sized M, weight-streaming GEMV for decode M."""
+import copy
+
 import numpy as np
 import pytest
 import torch
@@ -220,6 +222,78 @@ def test_loop_stack_open_more_than_eight_loops():
         torch.cuda.synchronize()
         linear_parity(y[t * M * lin.N:(t + 1) * M * lin.N].reshape(M, lin.N), xs[t], ol, t,
                       host(q8), host(s), layer.w_flips)
+
+
+def _slt_params(mp, T, seed):
+    """Loop-dependent copies of a module for SLT: per loop its own orthogonal
+    P1_t, P2_t and weight W_t (the shared weight plus a small loop-specific change)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for t in range(T):
+        q = copy.copy(mp)
+        a, b = mp.P1.shape[0], mp.P2.shape[0]
+        q.P1 = np.linalg.qr(rng.standard_normal((a, a)))[0].astype(np.float32)
+        q.P2 = np.linalg.qr(rng.standard_normal((b, b)))[0].astype(np.float32)
+        q.W = (mp.W + 0.002 * rng.standard_normal(mp.W.shape)).astype(np.float32)
+        out.append(q)
+    return out
+
+
+@pytest.mark.parametrize("wl,M,sel", [(synth.MLP, 256, 1), (synth.TINY, 64, 0)],
+                         ids=["mlp_up_selected", "tiny"])
+def test_loop_stack_slt_open(wl, M, sel):
+    """SLT serving in open mode: module `sel` has its own transform and weight at
+    every loop, the others share theirs (and keep sharing launches across loops);
+    every step is checked against the oracle's SLT schedule."""
+    params = synth.module_params(wl)
+    T, L = wl.T, len(wl.linears)
+    built = [make_layer(mp, wl.a_bits) for mp in params]
+    own = [make_layer(q, wl.a_bits) for q in _slt_params(params[sel], T, 7)]
+    tl = [[own[t] if l == sel else built[l] for l in range(L)] for t in range(T)]
+    xs, flat = _stack_inputs(wl, M)
+    xd = act_tensor(flat, wl.x_dtype)
+    y = host(lq.lq_loop_stack_slt(xd, [[h[0] for h in row] for row in tl], lq.LQ_OPEN, M=M))
+    torch.cuda.synchronize()
+    ys_or = O.loop_stack_slt_open(xs, [[h[1] for h in row] for row in tl], T)
+    off = 0
+    for t in range(T):
+        for l, lin in enumerate(wl.linears):
+            n = M * lin.N
+            yg = y[off:off + n].reshape(M, lin.N)
+            off += n
+            layer, ol = tl[t][l]
+            q8, _, sc = lq.lq_quantize_act(act_tensor(xs[t][l], wl.x_dtype), dev(ol.P1),
+                                           dev(ol.P2), float(ol.las[t]), wl.a_bits)
+            torch.cuda.synchronize()
+            y_or, _ = linear_parity(yg, xs[t][l], ol, t, host(q8), host(sc), layer.w_flips)
+            np.testing.assert_allclose(y_or, ys_or[t][l], rtol=1e-12, atol=0)
+
+
+def test_loop_stack_slt_chain_tiny():
+    """SLT serving in chain mode: the tiny shared linear selected, a different
+    transform and weight at each of its 4 loops, y_t feeding loop t + 1."""
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    (lin,) = wl.linears
+    own = [make_layer(q, 4) for q in _slt_params(mp, wl.T, 9)]
+    x0 = synth.loop_input(wl, lin, 0)
+    y = host(lq.lq_loop_stack_slt(dev(x0), [[h[0]] for h in own], lq.LQ_CHAIN, M=wl.M))
+    torch.cuda.synchronize()
+    ys = O.loop_stack_slt_chain(x0, [[h[1]] for h in own], wl.T)
+    for t in range(wl.T):
+        check_gemm(y[t * wl.M * lin.N:(t + 1) * wl.M * lin.N].reshape(wl.M, lin.N), ys[t][0],
+                   what=f"slt chain t={t}")
+
+
+def test_loop_stack_slt_rejects_shape_mismatch():
+    wl = synth.MLP
+    params = synth.module_params(wl)
+    gate, _ = make_layer(params[0], 4)
+    down, _ = make_layer(params[2], 4)
+    x = torch.zeros(2 * 64 * 2048, device="cuda")
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_loop_stack_slt(x, [[gate], [down]], lq.LQ_OPEN, M=64)
+    assert e.value.status == lq.LQ_ERR_SHAPE
 
 
 def test_loop_stack_chain_tiny():

@@ -293,6 +293,39 @@ def test_loop_driver_reductions():
     assert rel < 0.2
 
 
+def test_slt_schedule_reductions():
+    """SLT serving: with every loop mapped to the shared layer it is the plain
+    open / chain schedule; a loop-dependent layer at loop t gives, at that
+    step, exactly the single-layer result of that layer, and a loop-dependent
+    transform P_t with the weight folded by the same P_t still approximates
+    x W^T (Section 2, Eqs. (2)-(3): folding keeps the product up to
+    quantization), while a weight folded by another loop's transform does not."""
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    shared = O.OracleLayer(mp.W, mp.P1, mp.P2, mp.las, 4)
+    xs = [[synth.loop_input(wl, mp.lin, t)] for t in range(3)]
+    assert all(np.array_equal(a[0], b[0]) for a, b in
+               zip(O.loop_stack_slt_open(xs, [[shared]] * 3, 3), O.loop_stack_open(xs, [shared], 3)))
+    ch_a = O.loop_stack_slt_chain(xs[0][0], [[shared]] * 3, 3)
+    ch_b = O.loop_stack_chain(xs[0][0], [shared], 3)
+    assert all(np.array_equal(a[0], b[0]) for a, b in zip(ch_a, ch_b))
+    # loop 1 gets its own transform pair and the weight folded with it
+    rng = np.random.default_rng(5)
+    P1t = np.linalg.qr(rng.standard_normal((16, 16)))[0].astype(np.float32)
+    P2t = np.linalg.qr(rng.standard_normal((16, 16)))[0].astype(np.float32)
+    own = O.OracleLayer(mp.W, P1t, P2t, mp.las, 4)
+    ys = O.loop_stack_slt_open(xs, [[shared], [own], [shared]], 3)
+    assert np.array_equal(ys[1][0], own.forward(xs[1][0], 1))
+    assert np.array_equal(ys[0][0], shared.forward(xs[0][0], 0))
+    y_ref = xs[1][0].astype(np.float64) @ mp.W.astype(np.float64).T
+    rel = np.linalg.norm(ys[1][0] - y_ref) / np.linalg.norm(y_ref)
+    assert rel < 0.2
+    # mismatched pair: rotate with P_t but multiply the shared fold
+    mixed = O.OracleLayer(mp.W, P1t, P2t, mp.las, 4, Q1=shared.Q1, Q2=shared.Q2)
+    rel_bad = np.linalg.norm(mixed.forward(xs[1][0], 1) - y_ref) / np.linalg.norm(y_ref)
+    assert rel_bad > 0.5
+
+
 # ----------------------------------------------------------------------------
 # planted mistakes: a copy of the oracle with one plausible error must fail a pin
 # ----------------------------------------------------------------------------
