@@ -363,6 +363,35 @@ def aux_schedules(lq, torch, dev, stream, timed, wl, params, layers, x_dev, ops_
     out["loop_by_loop"] = {"ms_per_step": ms, "TOPS": ops_step / (ms * 1e-3) / 1e12,
                            "launches_per_step": 2 * T * L}
 
+    lins = wl.linears
+    if all(lins[l].N == lins[(l + 1) % L].K for l in range(L)):
+        # chain mode: loops strictly in sequence, y of each step feeding the next
+        # (inputs: the first step's x), plain and with CTA at the T - 1 transitions
+        x0 = x_dev[: M * lins[0].K]
+        run = lambda: lq.lq_loop_stack(x0, layers, T, lq.LQ_CHAIN, M=M, y=y, ws=ws1,
+                                       stream=stream)
+        for _ in range(3):
+            run()
+        ms = timed(n, run) / n
+        out["chain"] = {"ms_per_step": ms, "TOPS": ops_step / (ms * 1e-3) / 1e12}
+        d = lins[-1].N
+        rng = np.random.default_rng(23)
+        U = torch.from_numpy((0.05 * rng.standard_normal((d, 8))).astype(np.float32)).to(dev)
+        V = torch.from_numpy((0.05 * rng.standard_normal((d, 8))).astype(np.float32)).to(dev)
+        a = torch.from_numpy((1 + 0.1 * rng.standard_normal((T - 1, d))).astype(np.float32)).to(dev)
+        b = torch.from_numpy((0.1 * rng.standard_normal((T - 1, d))).astype(np.float32)).to(dev)
+        cta = lq.lq_cta_create(U, V, a, b, rng.uniform(0.1, 0.9, T - 1))
+        ws_c = torch.empty(lq.lq_cta_stack_workspace_bytes(layers, M), dtype=torch.uint8,
+                           device=dev)
+        run = lambda: lq.lq_loop_stack_cta(x0, layers, T, cta, M=M, y=y, ws=ws_c, stream=stream)
+        for _ in range(3):
+            run()
+        ms_c = timed(n, run) / n
+        out["chain_cta"] = {"ms_per_step": ms_c, "TOPS": ops_step / (ms_c * 1e-3) / 1e12,
+                            "transitions": T - 1,
+                            "us_per_transition": (ms_c - ms) * 1e3 / max(T - 1, 1)}
+        cta.free()
+
     rng = np.random.default_rng(17)
     own, keep = [], []
     for t in range(T):

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "liblq.so")
-SOURCES = ["lq_api.cu", "lq_quant.cu", "lq_gemm.cu", "lq_gemv.cu", "lq_noalloc.cu"]
+SOURCES = ["lq_api.cu", "lq_quant.cu", "lq_gemm.cu", "lq_gemv.cu", "lq_cta.cu", "lq_noalloc.cu"]
 HEADERS = ["lq_common.cuh"]
 
 NVCC_FLAGS = [

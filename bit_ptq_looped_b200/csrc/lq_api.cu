@@ -54,6 +54,18 @@ struct lq_layer {
   std::vector<float> las;
 };
 
+struct lq_cta {
+  uint64_t id = 0;
+  int64_t d = 0;
+  int rank = 0, n_trans = 0;
+  float* U8 = nullptr;  // device d x 8, columns >= rank zero
+  float* V8 = nullptr;  // device d x 8
+  float* a = nullptr;   // device n_trans x d
+  float* b = nullptr;   // device n_trans x d
+  std::vector<float> eta;
+  int device = 0;
+};
+
 namespace {
 
 std::atomic<uint64_t> g_layer_ids{1};
@@ -144,7 +156,9 @@ struct GraphKey {
   void* ws;
   int64_t ws_bytes;
   int device;
+  uint64_t cta = 0;
   bool operator<(const GraphKey& o) const {
+    if (cta != o.cta) return cta < o.cta;
     if (x != o.x) return x < o.x;
     if (dtype != o.dtype) return dtype < o.dtype;
     if (M != o.M) return M < o.M;
@@ -159,16 +173,25 @@ struct GraphKey {
 };
 
 std::mutex g_graph_mu;
-std::map<GraphKey, cudaGraphExec_t> g_graphs;
+struct CachedGraph {
+  cudaGraphExec_t exec;
+  uint64_t last_use;
+};
+std::map<GraphKey, CachedGraph> g_graphs;
+uint64_t g_graph_clock = 0;
+// at most this many instantiated schedules stay cached (the least recently
+// used goes first): callers that pass a new workspace or output buffer on
+// every call would otherwise grow the cache without bound
+constexpr size_t kMaxCachedGraphs = 64;
 std::map<int, cudaStream_t> g_capture_streams;
 
 void drop_graphs_of_layer(uint64_t id) {
   std::lock_guard<std::mutex> lk(g_graph_mu);
   for (auto it = g_graphs.begin(); it != g_graphs.end();) {
-    bool uses = false;
+    bool uses = it->first.cta == id;
     for (uint64_t l : it->first.layer_ids) uses |= (l == id);
     if (uses) {
-      cudaGraphExecDestroy(it->second);
+      cudaGraphExecDestroy(it->second.exec);
       it = g_graphs.erase(it);
     } else {
       ++it;
@@ -658,7 +681,7 @@ lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_l
 static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
                                const std::vector<const lq_layer*>& tl, int32_t L, int32_t T,
                                int32_t mode, float* d_y, void* d_ws, int64_t ws_bytes,
-                               cudaStream_t s) {
+                               cudaStream_t s, const lq_cta* cta = nullptr) {
   const size_t esz = x_dtype == LQ_BF16 ? 2 : 4;
   auto at = [&](int t, int l) { return tl[(size_t)t * L + l]; };
   if (mode == LQ_OPEN) {
@@ -697,6 +720,10 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
   }
   float* ycur = d_y;
   const float* prev_y = nullptr;
+  // CTA state (the adapted input of the next loop) after the codes and steps
+  int64_t codes_ws = 0;
+  for (const lq_layer* ly : tl) codes_ws = std::max(codes_ws, ws_bytes_for(M, ly->wq->K));
+  float* state = (float*)((char*)d_ws + round_up(codes_ws, 256));
   for (int t = 0; t < T; ++t) {
     for (int l = 0; l < L; ++l) {
       const lq_layer* ly = at(t, l);
@@ -710,6 +737,13 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
       prev_y = ycur;
       ycur += M * ly->wq->N;
     }
+    if (cta && t + 1 < T) {  // loop transition t -> t + 1
+      cudaError_t e = launch_cta_apply(prev_y, M, (int)cta->d, cta->U8, cta->V8,
+                                       cta->a + (size_t)t * cta->d, cta->b + (size_t)t * cta->d,
+                                       cta->eta[t], state, s, !probe_on());
+      if (e != cudaSuccess) return cuda_error(e, "cta launch");
+      prev_y = state;
+    }
   }
   return LQ_OK;
 }
@@ -718,7 +752,7 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
 static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
                                  const std::vector<const lq_layer*>& tl, int32_t L, int32_t T,
                                  int32_t mode, float* d_y, void* d_ws, int64_t ws_bytes,
-                                 void* stream) {
+                                 void* stream, const lq_cta* cta = nullptr) {
   if (mode != LQ_OPEN && mode != LQ_CHAIN) {
     set_error("unknown mode %d", mode);
     return LQ_ERR_ARG;
@@ -752,6 +786,22 @@ static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
       }
     }
   }
+  if (cta) {
+    if (mode != LQ_CHAIN) {
+      set_error("transition alignment needs chain mode");
+      return LQ_ERR_ARG;
+    }
+    if (cta->d != tl[L - 1]->wq->N) {
+      set_error("CTA width %lld != state width %lld", (long long)cta->d,
+                (long long)tl[L - 1]->wq->N);
+      return LQ_ERR_SHAPE;
+    }
+    if (cta->n_trans < T - 1) {
+      set_error("CTA has %d transitions, T=%d needs %d", cta->n_trans, T, T - 1);
+      return LQ_ERR_SHAPE;
+    }
+    need = round_up(need, 256) + round_up(M * cta->d * 4, 256);
+  }
   if (M == 0) return LQ_OK;
   if (!d_x || !d_y || !d_ws) {
     set_error("null pointer");
@@ -771,7 +821,7 @@ static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
   cudaError_t e = cudaStreamIsCapturing(s, &cap);
   if (e != cudaSuccess) return cuda_error(e, "stream query");
   if (cap != cudaStreamCaptureStatusNone || probe_on())
-    return enqueue_stack(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, s);
+    return enqueue_stack(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, s, cta);
 
   GraphKey key;
   key.x = d_x;
@@ -783,6 +833,7 @@ static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
   key.y = d_y;
   key.ws = d_ws;
   key.ws_bytes = ws_bytes;
+  key.cta = cta ? cta->id : 0;
   cudaGetDevice(&key.device);
 
   std::lock_guard<std::mutex> lk(g_graph_mu);
@@ -799,7 +850,7 @@ static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
     }
     if ((e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal)) != cudaSuccess)
       return cuda_error(e, "begin capture");
-    st = enqueue_stack(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, cs);
+    st = enqueue_stack(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, cs, cta);
     cudaGraph_t g = nullptr;
     e = cudaStreamEndCapture(cs, &g);
     if (st != LQ_OK) {
@@ -811,9 +862,18 @@ static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
     e = cudaGraphInstantiate(&ge, g, 0);
     cudaGraphDestroy(g);
     if (e != cudaSuccess) return cuda_error(e, "instantiate graph");
-    it = g_graphs.emplace(key, ge).first;
+    if (g_graphs.size() >= kMaxCachedGraphs) {
+      auto old = g_graphs.begin();
+      for (auto jt = g_graphs.begin(); jt != g_graphs.end(); ++jt)
+        if (jt->second.last_use < old->second.last_use) old = jt;
+      // a graph still running on some stream stays valid: destruction is deferred
+      cudaGraphExecDestroy(old->second.exec);
+      g_graphs.erase(old);
+    }
+    it = g_graphs.emplace(key, CachedGraph{ge, 0}).first;
   }
-  e = cudaGraphLaunch(it->second, s);
+  it->second.last_use = ++g_graph_clock;
+  e = cudaGraphLaunch(it->second.exec, s);
   if (e != cudaSuccess) return cuda_error(e, "graph launch");
   return LQ_OK;
 }
@@ -846,6 +906,123 @@ lq_status lq_loop_stack_slt(const void* d_x, int32_t x_dtype, int64_t M,
   }
   std::vector<const lq_layer*> tl(layers_tl, layers_tl + (size_t)T * L);
   return loop_stack_impl(d_x, x_dtype, M, tl, L, T, mode, d_y, d_ws, ws_bytes, stream);
+}
+
+lq_status lq_cta_create(const float* d_U, const float* d_V, int64_t d, int32_t rank,
+                        const float* d_a, const float* d_b, const float* h_eta, int32_t n_trans,
+                        lq_cta** out) {
+  if (!out || !d_U || !d_V || !d_a || !d_b || !h_eta) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  *out = nullptr;
+  if (d <= 0 || d > (1 << 24) || rank <= 0 || rank > 8 || n_trans <= 0) {
+    set_error("CTA needs d > 0, 1 <= rank <= 8 and at least one transition");
+    return LQ_ERR_ARG;
+  }
+  for (int t = 0; t < n_trans; ++t) {
+    if (!std::isfinite(h_eta[t])) {
+      set_error("gate %d is not finite", t);
+      return LQ_ERR_ARG;
+    }
+  }
+  lq_cta* c = new lq_cta();
+  c->d = d;
+  c->rank = rank;
+  c->n_trans = n_trans;
+  c->eta.assign(h_eta, h_eta + n_trans);
+  cudaGetDevice(&c->device);
+  const size_t b8 = (size_t)d * 8 * sizeof(float), bt = (size_t)n_trans * d * sizeof(float);
+  cudaError_t e = cudaMalloc(&c->U8, b8);
+  if (e == cudaSuccess) e = cudaMalloc(&c->V8, b8);
+  if (e == cudaSuccess) e = cudaMalloc(&c->a, bt);
+  if (e == cudaSuccess) e = cudaMalloc(&c->b, bt);
+  if (e == cudaSuccess) e = cudaMemset(c->U8, 0, b8);
+  if (e == cudaSuccess) e = cudaMemset(c->V8, 0, b8);
+  // caller's d x rank row-major factors into d x 8 rows
+  if (e == cudaSuccess)
+    e = cudaMemcpy2D(c->U8, 8 * sizeof(float), d_U, rank * sizeof(float), rank * sizeof(float),
+                     d, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy2D(c->V8, 8 * sizeof(float), d_V, rank * sizeof(float), rank * sizeof(float),
+                     d, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c->a, d_a, bt, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c->b, d_b, bt, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    lq_cta_free(c);
+    return cuda_error(e, "cta create");
+  }
+  c->id = g_layer_ids.fetch_add(1);
+  *out = c;
+  return LQ_OK;
+}
+
+void lq_cta_free(lq_cta* c) {
+  if (!c) return;
+  drop_graphs_of_layer(c->id);
+  cudaFree(c->U8);
+  cudaFree(c->V8);
+  cudaFree(c->a);
+  cudaFree(c->b);
+  delete c;
+}
+
+lq_status lq_cta_apply(const float* d_h, int64_t M, const lq_cta* cta, int32_t t, float* d_out,
+                       void* stream) {
+  if (!cta) {
+    set_error("null CTA");
+    return LQ_ERR_ARG;
+  }
+  if (M < 0) {
+    set_error("negative M");
+    return LQ_ERR_ARG;
+  }
+  if (t < 0 || t >= cta->n_trans) {
+    set_error("transition t=%d outside [0, %d)", t, cta->n_trans);
+    return LQ_ERR_SHAPE;
+  }
+  if (M == 0) return LQ_OK;
+  if (!d_h || !d_out) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_h) || !aligned16(d_out)) {
+    set_error("h and out must be 16-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  cudaError_t e = launch_cta_apply(d_h, M, (int)cta->d, cta->U8, cta->V8,
+                                   cta->a + (size_t)t * cta->d, cta->b + (size_t)t * cta->d,
+                                   cta->eta[t], d_out, (cudaStream_t)stream, false);
+  if (e != cudaSuccess) return cuda_error(e, "cta launch");
+  return LQ_OK;
+}
+
+int64_t lq_cta_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M) {
+  if (!layers || L <= 0 || M < 0 || !layers[L - 1]) return -1;
+  const int64_t base = lq_workspace_bytes(layers, L, M);
+  if (base < 0) return -1;
+  return round_up(base, 256) + round_up(M * layers[L - 1]->wq->N * 4, 256);
+}
+
+lq_status lq_loop_stack_cta(const void* d_x, int32_t x_dtype, int64_t M,
+                            const lq_layer* const* layers, int32_t L, int32_t T,
+                            const lq_cta* cta, float* d_y, void* d_ws, int64_t ws_bytes,
+                            void* stream) {
+  if (!layers || L <= 0 || T <= 0 || !cta) {
+    set_error("need layers, loops and a CTA");
+    return LQ_ERR_ARG;
+  }
+  for (int l = 0; l < L; ++l) {
+    if (layers[l] && layers[l]->T < T) {
+      set_error("layer %d has %d LAS clips but T=%d", l, layers[l]->T, T);
+      return LQ_ERR_SHAPE;
+    }
+  }
+  std::vector<const lq_layer*> tl((size_t)T * L);
+  for (int t = 0; t < T; ++t)
+    for (int l = 0; l < L; ++l) tl[(size_t)t * L + l] = layers[l];
+  return loop_stack_impl(d_x, x_dtype, M, tl, L, T, LQ_CHAIN, d_y, d_ws, ws_bytes, stream, cta);
 }
 
 lq_status lq_probe_enable(int32_t on) {

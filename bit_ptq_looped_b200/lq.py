@@ -12,6 +12,7 @@ import ctypes
 import os
 from typing import Optional, Sequence
 
+import numpy as np
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -49,6 +50,11 @@ SIGNATURES = {
     "lq_loop_linear": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack_slt": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
+    "lq_cta_create": (_i32, [_vp, _vp, _i64, _i32, _vp, _vp, _vp, _i32, _pp]),
+    "lq_cta_free": (None, [_vp]),
+    "lq_cta_apply": (_i32, [_vp, _i64, _vp, _i32, _vp, _vp]),
+    "lq_cta_stack_workspace_bytes": (_i64, [_pp, _i32, _i64]),
+    "lq_loop_stack_cta": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _vp, _vp, _vp, _i64, _vp]),
     "lq_check_device": (_i32, [_vp]),
     "lq_selftest_bounded_wait": (_i32, [_i64, _vp]),
     "lq_loop_linear_noalloc": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp]),
@@ -335,6 +341,74 @@ def lq_loop_stack_slt(x: torch.Tensor, layers_tl: Sequence[Sequence[Layer]], mod
     st = lib().lq_loop_stack_slt(_dev(x, "x"), dt, M, p, L, T, mode, _dev(y, "y"),
                                  _dev(ws, "ws"), ws.numel(), _stream(stream))
     _check(st, "lq_loop_stack_slt")
+    return y
+
+
+class Cta:
+    """Owner of an lq_cta handle (loop-transition adapter)."""
+
+    def __init__(self, handle: int, d: int, n_trans: int):
+        self.handle, self.d, self.n_trans = handle, d, n_trans
+
+    def free(self):
+        if self.handle:
+            lib().lq_cta_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def lq_cta_create(U: torch.Tensor, V: torch.Tensor, a: torch.Tensor, b: torch.Tensor,
+                  eta) -> Cta:
+    """U, V: d x r (r <= 8); a, b: n_trans x d (device float32); eta: n_trans gates."""
+    d, r = U.shape
+    n = a.shape[0]
+    eta_h = np.ascontiguousarray(np.asarray(eta, np.float32).reshape(n))
+    h = ctypes.c_void_p()
+    st = lib().lq_cta_create(_dev(U.contiguous(), "U"), _dev(V.contiguous(), "V"), d, r,
+                             _dev(a.contiguous(), "a"), _dev(b.contiguous(), "b"),
+                             eta_h.ctypes.data, n, ctypes.byref(h))
+    _check(st, "lq_cta_create")
+    return Cta(h.value, d, n)
+
+
+def lq_cta_apply(h: torch.Tensor, cta: Cta, t: int, *, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    M = h.shape[0]
+    if out is None:
+        out = torch.empty_like(h)
+    st = lib().lq_cta_apply(_dev(h, "h"), M, cta.handle, t, _dev(out, "out"), _stream(stream))
+    _check(st, "lq_cta_apply")
+    return out
+
+
+def lq_cta_stack_workspace_bytes(layers: Sequence[Layer], M: int) -> int:
+    p, keep = _layer_array(layers)
+    n = lib().lq_cta_stack_workspace_bytes(p, len(layers), M)
+    if n < 0:
+        raise ValueError("invalid layers")
+    return n
+
+
+def lq_loop_stack_cta(x: torch.Tensor, layers: Sequence[Layer], T: int, cta: Cta, *, M: int,
+                      y: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                      x_dtype: Optional[int] = None, stream=None) -> torch.Tensor:
+    """Chain mode with the adapter at every loop transition; y: the T*L unadapted outputs.
+    Pass the same y and ws on every call to replay the recorded schedule."""
+    if y is None:
+        y = torch.empty(T * M * sum(l.N for l in layers), dtype=torch.float32, device=x.device)
+    p, keep = _layer_array(layers)
+    if ws is None:
+        ws = torch.empty(max(lq_cta_stack_workspace_bytes(layers, M), 256), dtype=torch.uint8,
+                         device=x.device)
+    dt = _dtype_code(x) if x_dtype is None else x_dtype
+    st = lib().lq_loop_stack_cta(_dev(x, "x"), dt, M, p, len(layers), T, cta.handle,
+                                 _dev(y, "y"), _dev(ws, "ws"), ws.numel(), _stream(stream))
+    _check(st, "lq_loop_stack_cta")
     return y
 
 

@@ -67,6 +67,7 @@ typedef int32_t lq_status;
 
 typedef struct lq_wq lq_wq;        /* resident quantized weights (library-owned) */
 typedef struct lq_layer lq_layer;  /* weights + P factors + LAS clips of one module */
+typedef struct lq_cta lq_cta;      /* loop-transition adapter (CTA), library-owned */
 
 /* Thread-local text of the last error (empty string if none). */
 const char* lq_last_error(void);
@@ -235,6 +236,52 @@ lq_status lq_loop_stack(const void* d_x, int32_t x_dtype, int64_t M,
 lq_status lq_loop_stack_slt(const void* d_x, int32_t x_dtype, int64_t M,
                             const lq_layer* const* layers_tl, int32_t L, int32_t T, int32_t mode,
                             float* d_y, void* d_ws, int64_t ws_bytes, void* stream);
+
+/*
+ * Cross-loop transition alignment (CTA): an affine plus gated low-rank adapter
+ * applied to the recurrent state only at loop transitions
+ * ("paper_specification.yaml" of the LoopQ reproduction: cta, Section 4.3,
+ * Eq. (7); implementation_status lq5: U and V shared, a_t, b_t and the gate
+ * eta_t loop-dependent, rank 8, identity at initialization).  Eq. (7) is not
+ * printed on the pages; this library takes the plainest reading,
+ *     h' = a_t * h + b_t + eta_t * (h V) U^T,
+ * computed in float64 and rounded once to float32.
+ *
+ * lq_cta_create -- copy the adapter to library-owned device memory.
+ *   d_U, d_V  d x rank float32 row-major (device), 1 <= rank <= 8;
+ *   d_a, d_b  n_trans x d float32 row-major (device): a_t, b_t of transition t
+ *             (t -> t + 1);  h_eta[n_trans] (host, finite): the gates.
+ * Synchronous.  LQ_ERR_ARG on null pointers or bad sizes, LQ_ERR_CUDA on a
+ * failed copy or allocation.  Release with lq_cta_free.
+ */
+lq_status lq_cta_create(const float* d_U, const float* d_V, int64_t d, int32_t rank,
+                        const float* d_a, const float* d_b, const float* h_eta, int32_t n_trans,
+                        lq_cta** out);
+void lq_cta_free(lq_cta* cta);
+
+/*
+ * lq_cta_apply -- d_out = CTA_t(d_h) for M rows of width d (float32, row-major,
+ * 16-byte aligned; d_out may equal d_h).  LQ_ERR_SHAPE if t is not a
+ * transition of the adapter.  Asynchronous on `stream`.
+ */
+lq_status lq_cta_apply(const float* d_h, int64_t M, const lq_cta* cta, int32_t t, float* d_out,
+                       void* stream);
+
+/*
+ * lq_loop_stack_cta -- chain-mode lq_loop_stack with CTA at every loop
+ * transition: after loop t < T-1 the state passed to loop t + 1 is
+ * CTA_t(y_{t, L-1}).  d_y receives the unadapted outputs y_{t,l}, ordered
+ * (t, l) as in lq_loop_stack.  The adapter width must be N_{L-1} (= K_0) and
+ * it must have at least T - 1 transitions (LQ_ERR_SHAPE).  The workspace must
+ * hold lq_cta_stack_workspace_bytes(layers, L, M) bytes: the codes and steps
+ * plus the adapted state.  Graph reuse, programmatic launch and errors as
+ * lq_loop_stack.
+ */
+int64_t lq_cta_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M);
+lq_status lq_loop_stack_cta(const void* d_x, int32_t x_dtype, int64_t M,
+                            const lq_layer* const* layers, int32_t L, int32_t T,
+                            const lq_cta* cta, float* d_y, void* d_ws, int64_t ws_bytes,
+                            void* stream);
 
 /*
  * lq_loop_linear_noalloc -- lq_loop_linear for callers that cannot allocate

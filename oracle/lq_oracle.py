@@ -280,3 +280,46 @@ def loop_stack_slt_chain(x0: np.ndarray, layers_tl, T: int):
         ys.append(row)
     return ys
 
+
+# ----------------------------------------------------------------------------
+# cross-loop transition alignment (CTA) at loop transitions
+# ----------------------------------------------------------------------------
+def cta_apply(h: np.ndarray, a_t: np.ndarray, b_t: np.ndarray, eta_t: float,
+              U: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """CTA ("paper_specification.yaml" of the LoopQ reproduction: cta, Section
+    4.3, Eq. (7); implementation_status lq5): an affine plus gated low-rank
+    adapter applied only at loop transitions, U and V shared across
+    transitions, a_t, b_t and the gate eta_t loop-dependent; rank 8
+    (cta_rank); identity at initialization.  Eq. (7) itself is not printed on
+    the pages; the plainest reading of that description is taken:
+
+        h' = a_t * h + b_t + eta_t * (h V) U^T      (U, V: d x r; a_t, b_t: d)
+
+    computed in float64 and rounded once to float32 (the carried state is
+    float32)."""
+    h64 = np.asarray(h, np.float32).astype(np.float64)
+    p = h64 @ np.asarray(V, np.float32).astype(np.float64)            # M x r
+    low = p @ np.asarray(U, np.float32).astype(np.float64).T          # M x d
+    out = (np.asarray(a_t, np.float32).astype(np.float64)[None, :] * h64
+           + np.asarray(b_t, np.float32).astype(np.float64)[None, :]
+           + np.float64(np.float32(eta_t)) * low)
+    return out.astype(np.float32)
+
+
+def loop_stack_chain_cta(x0: np.ndarray, layers, T: int, a, b, eta, U, V):
+    """Chain mode with CTA at every transition: after loop t < T - 1 the state
+    that feeds loop t + 1 is cta_apply(y_{t, L-1}, a[t], b[t], eta[t]); the
+    outputs y_{t,l} themselves are returned unadapted."""
+    ys = []
+    cur = np.asarray(x0, np.float32)
+    for t in range(T):
+        row = []
+        for layer in layers:
+            y = loop_linear(cur, layer, t)
+            row.append(y)
+            cur = y.astype(np.float32)
+        if t + 1 < T:
+            cur = cta_apply(cur, a[t], b[t], eta[t], U, V)
+        ys.append(row)
+    return ys
+

@@ -109,6 +109,15 @@ def test_loop_entry_points_reject_bad_arguments(L):
                            None) == lq.LQ_ERR_ARG
     assert L.lq_workspace_bytes(None, 1, 4) == -1
     assert L.lq_stack_workspace_bytes(None, 1, 4, 4) == -1
+    assert L.lq_cta_stack_workspace_bytes(None, 1, 4) == -1
+    assert L.lq_loop_stack_cta(fake, lq.LQ_F32, 4, None, 1, 4, None, fake, fake, 1 << 20,
+                               None) == lq.LQ_ERR_ARG
+    assert L.lq_loop_stack_slt(fake, lq.LQ_F32, 4, None, 1, 4, lq.LQ_OPEN, fake, fake, 1 << 20,
+                               None) == lq.LQ_ERR_ARG
+    assert L.lq_cta_apply(fake, 4, None, 0, fake, None) == lq.LQ_ERR_ARG
+    out = ctypes.c_void_p()
+    assert L.lq_cta_create(None, fake, 16, 8, fake, fake, None, 1, ctypes.byref(out)) == \
+        lq.LQ_ERR_ARG
 
 
 def test_inverse_transpose_host_helper():

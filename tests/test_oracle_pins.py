@@ -326,6 +326,53 @@ def test_slt_schedule_reductions():
     assert rel_bad > 0.5
 
 
+def test_cta_pins():
+    """CTA (cta, Section 4.3, Eq. (7) as read: h' = a*h + b + eta*(h V) U^T):
+    identity at initialization, the affine part alone when the gate is 0, the
+    low-rank term against a brute-force sum in exact rationals, and a chained
+    schedule whose transition is the identity equals plain chain mode."""
+    rng = np.random.default_rng(3)
+    M, d, r = 5, 64, 8
+    h = rng.standard_normal((M, d)).astype(np.float32)
+    U = (0.1 * rng.standard_normal((d, r))).astype(np.float32)
+    V = (0.1 * rng.standard_normal((d, r))).astype(np.float32)
+    a = (1 + 0.1 * rng.standard_normal(d)).astype(np.float32)
+    b = (0.1 * rng.standard_normal(d)).astype(np.float32)
+    one, zero = np.ones(d, np.float32), np.zeros(d, np.float32)
+    assert np.array_equal(O.cta_apply(h, one, zero, 0.0, U, V), h)        # identity init
+    aff = (a.astype(np.float64) * h.astype(np.float64) + b).astype(np.float32)
+    assert np.array_equal(O.cta_apply(h, a, b, 0.0, U, V), aff)          # gate closed
+    # low-rank term in exact arithmetic: sum_r (sum_k h_k V_kr) U_jr
+    from fractions import Fraction
+    eta = np.float32(0.37)
+    got = O.cta_apply(h[:2, :16], one[:16], zero[:16], eta, U[:16], V[:16])
+    for m in range(2):
+        for j in range(16):
+            p = [sum(Fraction(float(h[m, k])) * Fraction(float(V[k, q])) for k in range(16))
+                 for q in range(r)]
+            exact = Fraction(float(h[m, j])) + Fraction(float(eta)) * sum(
+                p[q] * Fraction(float(U[j, q])) for q in range(r))
+            # one float32 rounding of a value computed to float64 accuracy
+            assert abs(float(got[m, j]) - float(exact)) <= 2 ** -23 * abs(float(exact)) + 1e-30
+    # with identity transitions the CTA schedule is the plain chain schedule
+    wl = synth.TINY
+    (mp,) = synth.module_params(wl)
+    layer = O.OracleLayer(mp.W, mp.P1, mp.P2, mp.las, 4)
+    x0 = synth.loop_input(wl, mp.lin, 0)
+    K = x0.shape[1]
+    ones, zeros = np.ones(K, np.float32), np.zeros(K, np.float32)
+    U0 = np.zeros((K, r), np.float32)
+    a_c = [ones] * 3
+    b_c = [zeros] * 3
+    c1 = O.loop_stack_chain_cta(x0, [layer], 4, a_c, b_c, [0.0] * 3, U0, U0)
+    c2 = O.loop_stack_chain(x0, [layer], 4)
+    assert all(np.array_equal(p[0], q[0]) for p, q in zip(c1, c2))
+    # a real transition changes the next loop's input and therefore its output
+    c3 = O.loop_stack_chain_cta(x0, [layer], 2, [a.repeat(4)[:K]] * 1, [b.repeat(4)[:K]] * 1,
+                                [0.5], np.tile(U, (4, 1)), np.tile(V, (4, 1)))
+    assert np.array_equal(c3[0][0], c2[0][0]) and not np.array_equal(c3[1][0], c2[1][0])
+
+
 # ----------------------------------------------------------------------------
 # planted mistakes: a copy of the oracle with one plausible error must fail a pin
 # ----------------------------------------------------------------------------
