@@ -58,8 +58,8 @@ struct lq_cta {
   uint64_t id = 0;
   int64_t d = 0;
   int rank = 0, n_trans = 0;
-  float* U8 = nullptr;  // device d x 8, columns >= rank zero
-  float* V8 = nullptr;  // device d x 8
+  double* U8 = nullptr;  // device d x 8 float64, columns >= rank zero
+  double* V8 = nullptr;  // device d x 8 float64
   float* a = nullptr;   // device n_trans x d
   float* b = nullptr;   // device n_trans x d
   std::vector<float> eta;
@@ -926,26 +926,36 @@ lq_status lq_cta_create(const float* d_U, const float* d_V, int64_t d, int32_t r
       return LQ_ERR_ARG;
     }
   }
+  if (d % 32) {
+    set_error("CTA width d=%lld must be a multiple of 32", (long long)d);
+    return LQ_ERR_SHAPE;
+  }
   lq_cta* c = new lq_cta();
   c->d = d;
   c->rank = rank;
   c->n_trans = n_trans;
   c->eta.assign(h_eta, h_eta + n_trans);
   cudaGetDevice(&c->device);
-  const size_t b8 = (size_t)d * 8 * sizeof(float), bt = (size_t)n_trans * d * sizeof(float);
-  cudaError_t e = cudaMalloc(&c->U8, b8);
+  // U, V to float64 d x 8 (zero columns past the rank), converted on the host
+  std::vector<float> hu((size_t)d * rank), hv((size_t)d * rank);
+  std::vector<double> u8((size_t)d * 8, 0.0), v8((size_t)d * 8, 0.0);
+  const size_t b8 = u8.size() * sizeof(double), bt = (size_t)n_trans * d * sizeof(float);
+  cudaError_t e = cudaMemcpy(hu.data(), d_U, hu.size() * sizeof(float), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(hv.data(), d_V, hv.size() * sizeof(float), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) {
+    for (int64_t k = 0; k < d; ++k)
+      for (int q = 0; q < rank; ++q) {
+        u8[k * 8 + q] = hu[k * rank + q];
+        v8[k * 8 + q] = hv[k * rank + q];
+      }
+  }
+  if (e == cudaSuccess) e = cudaMalloc(&c->U8, b8);
   if (e == cudaSuccess) e = cudaMalloc(&c->V8, b8);
   if (e == cudaSuccess) e = cudaMalloc(&c->a, bt);
   if (e == cudaSuccess) e = cudaMalloc(&c->b, bt);
-  if (e == cudaSuccess) e = cudaMemset(c->U8, 0, b8);
-  if (e == cudaSuccess) e = cudaMemset(c->V8, 0, b8);
-  // caller's d x rank row-major factors into d x 8 rows
-  if (e == cudaSuccess)
-    e = cudaMemcpy2D(c->U8, 8 * sizeof(float), d_U, rank * sizeof(float), rank * sizeof(float),
-                     d, cudaMemcpyDeviceToDevice);
-  if (e == cudaSuccess)
-    e = cudaMemcpy2D(c->V8, 8 * sizeof(float), d_V, rank * sizeof(float), rank * sizeof(float),
-                     d, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c->U8, u8.data(), b8, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c->V8, v8.data(), b8, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(c->a, d_a, bt, cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(c->b, d_b, bt, cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();

@@ -341,8 +341,8 @@ cudaError_t launch_group_gemm(const uint8_t* A, const float* sa, const uint8_t* 
 lq_status read_and_clear_device_status(cudaStream_t s);
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
 
-// CTA (lq_cta.cu): U8, V8 are d x 8 (rank padded with zero columns)
-cudaError_t launch_cta_apply(const float* h, int64_t M, int d, const float* U8, const float* V8,
+// CTA (lq_cta.cu): U8, V8 are float64 d x 8 (rank padded with zero columns), d % 32 == 0
+cudaError_t launch_cta_apply(const float* h, int64_t M, int d, const double* U8, const double* V8,
                              const float* a, const float* b, float eta, float* out,
                              cudaStream_t s, bool pdl);
 

@@ -64,6 +64,13 @@ def test_cta_apply_in_place_and_identity():
     assert e.value.status == lq.LQ_ERR_SHAPE
 
 
+def test_cta_create_rejects_width_not_multiple_of_32():
+    U, V, a, b, eta = _adapter(48, 8, 1, seed=8)
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_cta_create(dev(U), dev(V), dev(a), dev(b), eta)
+    assert e.value.status == lq.LQ_ERR_SHAPE
+
+
 def _tiny_layer():
     from tests.test_gpu_linear import make_layer
     wl = synth.TINY
