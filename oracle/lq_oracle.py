@@ -323,3 +323,22 @@ def loop_stack_chain_cta(x0: np.ndarray, layers, T: int, a, b, eta, U, V):
         ys.append(row)
     return ys
 
+
+# ----------------------------------------------------------------------------
+# trajectory Hessian accumulation (calibration statistic)
+# ----------------------------------------------------------------------------
+def trajectory_hessian(xs) -> np.ndarray:
+    """H = sum_t X_t^T X_t over the inputs X_t (M x K) a module sees at each
+    loop t ("Quantizing Looped Transformers: Feedback Exposure and Calibration
+    Blindness", Appendix Table 19: H_t = X_t^T X_t per recurrence step;
+    abstract and Section 5: accumulating the GPTQ Hessian across recurrence
+    steps instead of the step-0 activations alone).  Unnormalised (the
+    row-normalised form of Figure 5, 2 X^T X / m, is a scalar multiple);
+    float64."""
+    K = np.asarray(xs[0]).shape[1]
+    H = np.zeros((K, K), np.float64)
+    for x in xs:
+        x64 = np.asarray(x, np.float32).astype(np.float64)
+        H += x64.T @ x64
+    return H
+

@@ -373,6 +373,30 @@ def test_cta_pins():
     assert np.array_equal(c3[0][0], c2[0][0]) and not np.array_equal(c3[1][0], c2[1][0])
 
 
+def test_trajectory_hessian_pins():
+    """H = sum_t X_t^T X_t: brute force over (t, m, i, j) in exact rationals on
+    a tiny case, symmetry and positive semi-definiteness, T = 1 gives X^T X,
+    doubling the inputs quadruples H, and the sum over steps is the Hessian of
+    the concatenated steps."""
+    from fractions import Fraction
+    rng = np.random.default_rng(4)
+    xs = [synth.round_bf16(rng.standard_normal((3, 4)).astype(np.float32)) for _ in range(2)]
+    H = O.trajectory_hessian(xs)
+    for i in range(4):
+        for j in range(4):
+            exact = sum(Fraction(float(x[m, i])) * Fraction(float(x[m, j]))
+                        for x in xs for m in range(3))
+            assert H[i, j] == float(exact)  # bf16 products and these sums are exact in f64
+    big = [synth.round_bf16(rng.standard_normal((50, 32)).astype(np.float32)) for _ in range(3)]
+    Hb = O.trajectory_hessian(big)
+    assert np.array_equal(Hb, Hb.T)
+    assert np.linalg.eigvalsh(Hb).min() > -1e-9 * np.abs(Hb).max()
+    x0 = big[0].astype(np.float64)
+    assert np.allclose(O.trajectory_hessian(big[:1]), x0.T @ x0, rtol=0, atol=1e-12)
+    assert np.allclose(O.trajectory_hessian([2 * x for x in big]), 4 * Hb, rtol=1e-15, atol=0)
+    assert np.allclose(O.trajectory_hessian([np.concatenate(big)]), Hb, rtol=1e-13, atol=1e-12)
+
+
 # ----------------------------------------------------------------------------
 # planted mistakes: a copy of the oracle with one plausible error must fail a pin
 # ----------------------------------------------------------------------------
