@@ -392,6 +392,32 @@ def aux_schedules(lq, torch, dev, stream, timed, wl, params, layers, x_dev, ops_
                             "us_per_transition": (ms_c - ms) * 1e3 / max(T - 1, 1)}
         cta.free()
 
+    # trajectory Hessian of the first module over its T loop inputs (bf16)
+    lin0 = lins[0]
+    if wl.x_dtype == "bf16" and lin0.K % 128 == 0:
+        K0 = lin0.K
+        xh = torch.empty(T * M * K0, dtype=torch.bfloat16, device=dev)
+        off = 0
+        for t in range(T):  # loop t's input of module 0 inside the open-mode buffer
+            src = x_dev[(t * sum(l.K for l in lins)) * M: (t * sum(l.K for l in lins) + K0) * M]
+            xh[off: off + M * K0] = src
+            off += M * K0
+        Hh = torch.empty((K0, K0), dtype=torch.float32, device=dev)
+        wsh = torch.empty(lq.lib().lq_hessian_workspace_bytes(M, K0, T), dtype=torch.uint8,
+                          device=dev)
+        run = lambda: lq.lq_trajectory_hessian(xh, T, M=M, H=Hh, ws=wsh, stream=stream)
+        for _ in range(3):
+            run()
+        ms_h = timed(n, run) / n
+        flops = T * M * K0 * (K0 + 1)  # the symmetric product: one multiply-add per pair i <= j
+        peaks = load_peaks()
+        out["trajectory_hessian"] = {
+            "workload": f"H = sum_t X_t^T X_t, T={T} x {M} x {K0} bf16 -> {K0}x{K0} fp32",
+            "us": ms_h * 1e3, "TFLOP_s": flops / (ms_h * 1e-3) / 1e12,
+            "frac_bf16_peak": flops / (ms_h * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "flops": flops, "includes": "bf16 transpose of the inputs (one launch) + the product"}
+        del xh, Hh, wsh
+
     rng = np.random.default_rng(17)
     own, keep = [], []
     for t in range(T):

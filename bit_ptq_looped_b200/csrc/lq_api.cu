@@ -1035,6 +1035,69 @@ lq_status lq_loop_stack_cta(const void* d_x, int32_t x_dtype, int64_t M,
   return loop_stack_impl(d_x, x_dtype, M, tl, L, T, LQ_CHAIN, d_y, d_ws, ws_bytes, stream, cta);
 }
 
+int64_t lq_hessian_workspace_bytes(int64_t M, int64_t K, int32_t T) {
+  if (M < 0 || K <= 0 || T <= 0) return -1;
+  return round_up(K * hessian_rows_padded(M * T) * 2, 256);
+}
+
+lq_status lq_trajectory_hessian(const void* d_X, int32_t x_dtype, int64_t M, int64_t K,
+                                int32_t T, float* d_H, int32_t accumulate, void* d_ws,
+                                int64_t ws_bytes, void* stream) {
+  if (x_dtype != LQ_BF16) {
+    set_error("the trajectory Hessian takes bf16 inputs (products exact in float32)");
+    return LQ_ERR_UNSUPPORTED;
+  }
+  if (M < 0 || K <= 0 || T <= 0) {
+    set_error("invalid shape M=%lld K=%lld T=%d", (long long)M, (long long)K, T);
+    return LQ_ERR_ARG;
+  }
+  if (K % 128 || K > 65536) {
+    set_error("K=%lld must be a multiple of 128 and at most 65536", (long long)K);
+    return LQ_ERR_SHAPE;
+  }
+  if (!d_H) {
+    set_error("null H");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_H)) {
+    set_error("H must be 16-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  if (M == 0) {  // no rows: H = 0, or unchanged when accumulating
+    if (accumulate) return LQ_OK;
+    cudaError_t e = cudaMemsetAsync(d_H, 0, (size_t)K * K * sizeof(float), s);
+    return e == cudaSuccess ? LQ_OK : cuda_error(e, "clear H");
+  }
+  if (!d_X || !d_ws) {
+    set_error("null pointer");
+    return LQ_ERR_ARG;
+  }
+  if (!aligned16(d_X) || ((uintptr_t)d_ws & 255u)) {
+    set_error("X must be 16-byte aligned and the workspace 256-byte aligned");
+    return LQ_ERR_ALIGN;
+  }
+  if (M * T > ((int64_t)1 << 31) - 64) {
+    set_error("too many rows");
+    return LQ_ERR_SHAPE;
+  }
+  if (ws_bytes < lq_hessian_workspace_bytes(M, K, T)) {
+    set_error("workspace too small");
+    return LQ_ERR_WORKSPACE;
+  }
+  const char* why = nullptr;
+  cudaError_t e = launch_trajectory_hessian((const uint16_t*)d_X, M * T, K, (uint16_t*)d_ws, d_H,
+                                            accumulate ? 1 : 0, s, &why);
+  if (e != cudaSuccess) {
+    if (why) {
+      set_error("trajectory Hessian: %s", why);
+      return LQ_ERR_CUDA;
+    }
+    return cuda_error(e, "trajectory Hessian launch");
+  }
+  return LQ_OK;
+}
+
 lq_status lq_probe_enable(int32_t on) {
   std::lock_guard<std::mutex> lk(g_probe.mu);
   g_probe.on = on != 0;

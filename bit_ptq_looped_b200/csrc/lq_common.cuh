@@ -346,6 +346,13 @@ cudaError_t launch_cta_apply(const float* h, int64_t M, int d, const double* U8,
                              const float* a, const float* b, float eta, float* out,
                              cudaStream_t s, bool pdl);
 
+// trajectory Hessian (lq_gemm.cu): X is R x K bf16; Xt scratch of K x
+// hessian_rows_padded(R) bf16; K a multiple of 128; H K x K float32
+int64_t hessian_rows_padded(int64_t R);
+cudaError_t launch_trajectory_hessian(const uint16_t* X, int64_t R, int64_t K, uint16_t* Xt,
+                                      float* H, int accumulate, cudaStream_t s,
+                                      const char** why);
+
 // GEMV (lq_gemv.cu)
 // qa: activation codes in the kOpGemvAct layout, asum their group sums
 cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa,

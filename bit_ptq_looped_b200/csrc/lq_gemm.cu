@@ -430,6 +430,245 @@ __global__ void k_wait_selftest(uint64_t limit_ns) {
 }
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Trajectory Hessian H (+)= sum_t X_t^T X_t ("Quantizing Looped Transformers:
+// Feedback Exposure and Calibration Blindness", Appendix Table 19, H_t =
+// X_t^T X_t; accumulating the GPTQ Hessian across recurrence steps).
+//
+// The T loop inputs (bf16, R = T*M rows of K) are first transposed to Xt
+// (K x R_pad, R_pad = R rounded up to 64, zero padded), so that the reduction
+// index is contiguous.  Then H = Xt Xt^T on the tensor cores: one CTA per
+// 128 x 128 tile of the upper triangle (the lower one is its mirror), a TMA
+// warp streaming 128 x 64 bf16 tiles of both row blocks through a 6-stage
+// ring, an MMA warp issuing four kind::f16 MMAs (K = 16 each) per stage into
+// one float32 TMEM accumulator that runs over the whole reduction, and four
+// epilogue warps writing the tile and, off the diagonal, its transpose.
+// bf16 products are exact in float32; the sums are the tensor core's float32
+// accumulation.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int HT = 128;               // tile rows / columns of H
+constexpr int HK = 64;                // reduction elements per stage (128-byte bf16 rows)
+constexpr int H_STAGES = 6;
+constexpr uint32_t H_TILE_BYTES = HT * HK * 2;  // 16 KB
+constexpr uint32_t H_STAGE_TX = 2 * H_TILE_BYTES;
+constexpr int H_EPI_WARPS = 4;
+constexpr int H_WARP_TMA = H_EPI_WARPS, H_WARP_MMA = H_EPI_WARPS + 1;
+constexpr int H_THREADS = 32 * (H_EPI_WARPS + 2);
+constexpr uint32_t H_OFF_A = 0;
+constexpr uint32_t H_OFF_B = H_OFF_A + H_STAGES * H_TILE_BYTES;
+constexpr uint32_t H_OFF_BAR = H_OFF_B + H_STAGES * H_TILE_BYTES;
+constexpr uint32_t H_N_BARS = 2 * H_STAGES + 2;  // full, empty, accumulator full, drain
+constexpr uint32_t H_OFF_MISC = H_OFF_BAR + H_N_BARS * 8;
+constexpr uint32_t H_SMEM_BYTES = H_OFF_MISC + 16 + 1024;
+
+__host__ __device__ constexpr uint32_t instr_desc_bf16() {
+  // F32 accumulator, A and B bf16, both K-major, N = M = 128
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(HT >> 3) << 17) |
+         ((uint32_t)(HT >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// tile index of the upper triangle (row-major over mb <= nb) -> (mb, nb)
+__device__ __forceinline__ void upper_tile(int t, int nt, int& mb, int& nb) {
+  mb = 0;
+  while (t >= nt - mb) {
+    t -= nt - mb;
+    ++mb;
+  }
+  nb = mb + t;
+}
+
+__global__ void __launch_bounds__(H_THREADS, 1)
+    k_hessian(const __grid_constant__ CUtensorMap tmX, float* __restrict__ H, int K, int n_kb,
+              int accumulate) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_full = base + H_OFF_BAR;
+  const uint32_t bar_empty = bar_full + H_STAGES * 8;
+  const uint32_t bar_accf = bar_empty + H_STAGES * 8;
+  const uint32_t bar_drain = bar_accf + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + H_OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + H_OFF_MISC + 4);
+  const int nt = K / HT;
+  int mb, nb;
+  upper_tile(blockIdx.x, nt, mb, nb);
+  const int m0 = mb * HT, n0 = nb * HT;
+
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < H_STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_accf, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == H_WARP_TMA && lane == 0) prefetch_tmap(&tmX);
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), HT);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == H_WARP_TMA) {
+    if (lane == 0) {
+      pdl_wait();  // Xt comes from the transpose kernel
+      int issued = 0;
+      for (int kb = 0; kb < n_kb; ++kb) {
+        const int st = kb % H_STAGES;
+        const uint32_t ph = (uint32_t)(kb / H_STAGES) & 1u;
+        if (!mbar_wait_bounded(bar_empty + 8 * st, ph ^ 1u, abort_flag, &g_gemm_status,
+                               kWaitLimitNs))
+          break;
+        const uint32_t full = bar_full + 8 * st;
+        mbar_arrive_expect_tx(full, H_STAGE_TX);
+        tma_load_2d(base + H_OFF_A + st * H_TILE_BYTES, &tmX, full, kb * HK, m0);
+        tma_load_2d(base + H_OFF_B + st * H_TILE_BYTES, &tmX, full, kb * HK, n0);
+        issued = kb + 1;
+      }
+      for (int kb = max(0, issued - H_STAGES); kb < issued; ++kb)
+        mbar_wait_drain(bar_full + 8 * (kb % H_STAGES), (uint32_t)(kb / H_STAGES) & 1u);
+    }
+  } else if (warp == H_WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc_bf16();
+      bool ok = true;
+      for (int kb = 0; kb < n_kb; ++kb) {
+        const int st = kb % H_STAGES;
+        if (!mbar_wait_bounded(bar_full + 8 * st, (uint32_t)(kb / H_STAGES) & 1u, abort_flag,
+                               &g_gemm_status, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_st = base + H_OFF_A + st * H_TILE_BYTES;
+        const uint32_t b_st = base + H_OFF_B + st * H_TILE_BYTES;
+#pragma unroll
+        for (int j = 0; j < HK / 16; ++j)  // K = 16 bf16 = 32 bytes per MMA
+          umma_bf16(tmem_base, sw128_kmajor_desc(a_st + 32u * j),
+                    sw128_kmajor_desc(b_st + 32u * j), idesc, (kb | j) != 0 ? 1u : 0u);
+        umma_commit(bar_empty + 8 * st);
+      }
+      if (ok) umma_commit(bar_accf);
+      umma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0u);
+    }
+  } else {
+    // ---- epilogue: warp q reads TMEM lanes 32q..32q+31 = rows m0 + 32q + lane
+    const int q = warp;
+    const int row = q * 32 + lane;
+    pdl_wait();  // H may be read by an earlier kernel of the stream
+    if (mbar_wait_bounded(bar_accf, 0u, abort_flag, &g_gemm_status, kWaitLimitNs)) {
+      tc_fence_after();
+      const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < HT / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(lane_base + (uint32_t)(32 * c), r);
+        tmem_wait_ld();
+        // tile (m0 + row, n0 + 32c + i): each thread writes 32 consecutive floats of its row
+        float* dst = H + (size_t)(m0 + row) * K + n0 + 32 * c;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          float4 v = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                 __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+          if (accumulate) {
+            const float4 o = *reinterpret_cast<const float4*>(dst + i);
+            v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+          }
+          *reinterpret_cast<float4*>(dst + i) = v;
+        }
+        if (nb != mb) {
+          // mirrored tile (n0 + 32c + i, m0 + row): for each i the 32 lanes write 32
+          // consecutive floats
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float* md = H + (size_t)(n0 + 32 * c + i) * K + m0 + row;
+            float v = __uint_as_float(r[i]);
+            if (accumulate) v += *md;
+            *md = v;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, HT);
+  }
+}
+
+// X (R x K bf16, row-major) -> Xt (K x Rp, zero columns past R)
+__global__ void k_transpose_bf16(const uint16_t* __restrict__ X, int64_t R, int64_t K,
+                                 int64_t Rp, uint16_t* __restrict__ Xt) {
+  __shared__ uint16_t tile[64][66];
+  pdl_trigger();
+  const int64_t r0 = (int64_t)blockIdx.x * 64, k0 = (int64_t)blockIdx.y * 64;
+  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 256 threads: 64 x 4
+  for (int i = ty; i < 64; i += 4) {
+    const int64_t r = r0 + i, k = k0 + tx;
+    tile[i][tx] = (r < R && k < K) ? X[r * K + k] : (uint16_t)0;
+  }
+  __syncthreads();
+  pdl_wait();  // the previous kernel may still read Xt
+  for (int i = ty; i < 64; i += 4) {
+    const int64_t k = k0 + i, r = r0 + tx;
+    if (k < K && r < Rp) Xt[k * Rp + r] = tile[tx][i];
+  }
+}
+
+}  // namespace
+
+int64_t hessian_rows_padded(int64_t R) { return (R + HK - 1) / HK * HK; }
+
+cudaError_t launch_trajectory_hessian(const uint16_t* X, int64_t R, int64_t K, uint16_t* Xt,
+                                      float* H, int accumulate, cudaStream_t s,
+                                      const char** why) {
+  const int64_t Rp = hessian_rows_padded(R);
+  dim3 tg((unsigned)((Rp + 63) / 64), (unsigned)((K + 63) / 64));
+  cudaError_t e = launch_kernel(k_transpose_bf16, tg, dim3(256), 0, s, false, X, R, K, Rp, Xt);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mX;
+  if (!make_map_2d(&mX, Xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Rp, K, Rp * 2, HK, HT,
+                   CU_TENSOR_MAP_SWIZZLE_128B)) {
+    if (why) *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  static uint64_t attr_set_mask = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!((attr_set_mask >> (dev & 63)) & 1u)) {
+    e = cudaFuncSetAttribute(k_hessian, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)H_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set_mask |= 1ull << (dev & 63);
+  }
+  const int nt = (int)(K / HT);
+  return launch_kernel(k_hessian, dim3((unsigned)(nt * (nt + 1) / 2)), dim3(H_THREADS),
+                       H_SMEM_BYTES, s, true, mX, H, (int)K, (int)(Rp / HK), accumulate);
+}
+
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s) {
   k_wait_selftest<<<1, 32, 0, s>>>(limit_ns);
   return cudaGetLastError();

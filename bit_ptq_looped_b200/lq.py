@@ -50,6 +50,8 @@ SIGNATURES = {
     "lq_loop_linear": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
     "lq_loop_stack_slt": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _i32, _vp, _vp, _i64, _vp]),
+    "lq_hessian_workspace_bytes": (_i64, [_i64, _i64, _i32]),
+    "lq_trajectory_hessian": (_i32, [_vp, _i32, _i64, _i64, _i32, _vp, _i32, _vp, _i64, _vp]),
     "lq_cta_create": (_i32, [_vp, _vp, _i64, _i32, _vp, _vp, _vp, _i32, _pp]),
     "lq_cta_free": (None, [_vp]),
     "lq_cta_apply": (_i32, [_vp, _i64, _vp, _i32, _vp, _vp]),
@@ -342,6 +344,26 @@ def lq_loop_stack_slt(x: torch.Tensor, layers_tl: Sequence[Sequence[Layer]], mod
                                  _dev(ws, "ws"), ws.numel(), _stream(stream))
     _check(st, "lq_loop_stack_slt")
     return y
+
+
+def lq_trajectory_hessian(x: torch.Tensor, T: int, *, M: int, H: Optional[torch.Tensor] = None,
+                          accumulate: bool = False, ws: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """x: the T loop inputs back to back (T*M x K bf16); returns H (K x K float32),
+    H = sum_t X_t^T X_t, or H + that sum with accumulate=True."""
+    K = x.numel() // max(T * M, 1) if x.dim() == 1 else x.shape[-1]
+    if H is None:
+        H = torch.zeros((K, K), dtype=torch.float32, device=x.device)
+    if ws is None:
+        n = lib().lq_hessian_workspace_bytes(M, K, T)
+        if n < 0:
+            raise ValueError("invalid shape")
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=x.device)
+    st = lib().lq_trajectory_hessian(_dev(x, "x"), _dtype_code(x), M, K, T, _dev(H, "H"),
+                                     1 if accumulate else 0, _dev(ws, "ws"), ws.numel(),
+                                     _stream(stream))
+    _check(st, "lq_trajectory_hessian")
+    return H
 
 
 class Cta:

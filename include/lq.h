@@ -285,6 +285,27 @@ lq_status lq_loop_stack_cta(const void* d_x, int32_t x_dtype, int64_t M,
                             void* stream);
 
 /*
+ * lq_trajectory_hessian -- calibration statistic of one module over its loop
+ * inputs: H = sum_t X_t^T X_t (or H += that sum when `accumulate` is set),
+ * the Hessian accumulated across recurrence steps ("Quantizing Looped
+ * Transformers: Feedback Exposure and Calibration Blindness", Appendix Table
+ * 19, H_t = X_t^T X_t; abstract and Section 5, accumulating the GPTQ Hessian
+ * across recurrence steps).  Unnormalised.
+ *   d_X   T inputs back to back, each M x K bf16 row-major (x_dtype LQ_BF16;
+ *         others LQ_ERR_UNSUPPORTED), 16-byte aligned;
+ *   d_H   K x K float32 row-major (read when accumulating);
+ *   d_ws  lq_hessian_workspace_bytes(M, K, T) bytes, 256-byte aligned
+ *         (the transposed inputs).
+ * K must be a multiple of 128 (LQ_ERR_SHAPE).  bf16 products are exact in
+ * float32; the sums are the tensor cores' float32 accumulation over M*T terms.
+ * Asynchronous on `stream`.
+ */
+int64_t lq_hessian_workspace_bytes(int64_t M, int64_t K, int32_t T);
+lq_status lq_trajectory_hessian(const void* d_X, int32_t x_dtype, int64_t M, int64_t K,
+                                int32_t T, float* d_H, int32_t accumulate, void* d_ws,
+                                int64_t ws_bytes, void* stream);
+
+/*
  * lq_loop_linear_noalloc -- lq_loop_linear for callers that cannot allocate
  * device memory, so cannot provide its workspace: for instance the enqueue
  * hook of another runtime that hands over only input and output buffers, a
