@@ -44,8 +44,8 @@ def _check(Hg, xs, H0=None, rows=None):
         A = A + np.abs(H0)
     err = np.abs(Hg.astype(np.float64) - Hor)
     assert np.all(err <= n * 2.0 ** -22 * A + 1e-30), err.max()
-    rel = np.linalg.norm(err) / np.linalg.norm(Hor)
-    assert rel < 1e-5, rel
+    # and on average far inside that bound (a random walk of float32 roundings)
+    assert np.linalg.norm(err) <= 16 * np.sqrt(n) * 2.0 ** -24 * np.linalg.norm(A)
 
 
 @pytest.mark.parametrize("M,K,T", [(64, 256, 4), (1024, 1024, 2), (100, 384, 3), (1, 128, 1)])
