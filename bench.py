@@ -309,7 +309,7 @@ def aux_hbm_kernels(lq, torch, dev, stream, timed, peaks):
     for w in wqs:
         w.free()
     del x, y, ws
-    # the GEMV kernel's streaming rate on one large launch: W4A8, M = 4, K = 2048,
+    # the GEMV kernel's streaming rate on one large launch: W4A8, M = 1, 4, 16, K = 2048,
     # N = 36 x 5632 weight rows (263 MB packed, > 2x L2), seeded N(0, 0.02) weights
     Nb = 36 * 5632
     g = torch.Generator(device=dev)
@@ -320,26 +320,28 @@ def aux_hbm_kernels(lq, torch, dev, stream, timed, peaks):
     wqb = lq.lq_pack_weights(Wf)
     del Wf
     lb = lq.lq_layer_create(wqb, P1, P2, mp.las, 8)
-    xb = torch.from_numpy(synth.loop_input(wl, wl.linears[0], 0)).to(torch.bfloat16).to(dev)
-    yb = torch.empty((Md, Nb), dtype=torch.float32, device=dev)
-    wsb = lq.workspace([lb], Md, dev)
+    for Ms in (1, 4, 16):  # decode row counts of the decode configuration
+        xb = torch.from_numpy(synth.loop_input(synth.decode_workload(Ms, 5632, 8),
+                                               wl.linears[0], 0)).to(torch.bfloat16).to(dev)
+        yb = torch.empty((Ms, Nb), dtype=torch.float32, device=dev)
+        wsb = lq.workspace([lb], Ms, dev)
 
-    def b_step():
-        lq.lq_loop_linear(xb, lb, 0, y=yb, ws=wsb, stream=stream)
+        def b_step():
+            lq.lq_loop_linear(xb, lb, 0, y=yb, ws=wsb, stream=stream)
 
-    for _ in range(3):
-        b_step()
-    lq.lq_probe_enable(True)
-    timed(10, b_step, flush_between=False)
-    pr = lq.lq_probe_read()
-    lq.lq_probe_enable(False)
-    gemv_ms, gemv_n = pr["gemv"]
-    avg = gemv_ms / max(gemv_n, 1)
-    byts = Nb * 2048 // 2 + Nb * 64 * 4 + Md * 2048 + Md * 64 * 8 + Md * Nb * 4
-    out["gemv_stream"] = {
-        "workload": f"W4A8 M={Md} K=2048 N={Nb}, one launch", "us": avg * 1e3,
-        "bytes_per_launch": byts, "GB_s": byts / (avg * 1e-3) / 1e9,
-        "frac_hbm": byts / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        for _ in range(3):
+            b_step()
+        lq.lq_probe_enable(True)
+        timed(10, b_step, flush_between=False)
+        pr = lq.lq_probe_read()
+        lq.lq_probe_enable(False)
+        gemv_ms, gemv_n = pr["gemv"]
+        avg = gemv_ms / max(gemv_n, 1)
+        byts = Nb * 2048 // 2 + Nb * 64 * 4 + Ms * 2048 + Ms * 64 * 8 + Ms * Nb * 4
+        out["gemv_stream" if Ms == 4 else f"gemv_stream_M{Ms}"] = {
+            "workload": f"W4A8 M={Ms} K=2048 N={Nb}, one launch", "us": avg * 1e3,
+            "bytes_per_launch": byts, "GB_s": byts / (avg * 1e-3) / 1e9,
+            "frac_hbm": byts / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     lb.free()
     wqb.free()
     return out

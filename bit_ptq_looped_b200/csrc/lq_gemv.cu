@@ -231,10 +231,18 @@ cudaError_t launch_mb(const int8_t* qa, const int* asum, const float* sa, const 
   const int64_t G = K / kGroup;
   if (G > 128) return launch_rpw<MB, 8, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
   if (G > 64) return launch_rpw<MB, 4, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  // up to 4 rows: three weight rows per warp once that still gives every SM
-  // one and a half blocks (16 rows keep one: their partial sums need the registers)
-  if (MB <= 4 && N >= (int64_t)num_sms() * kGemvWarps * 3 * 3 / 2)
-    return launch_rpw<MB, 2, (MB <= 4 ? 3 : 1)>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  // up to 4 rows (16 rows keep one: their partial sums need the registers):
+  // when one resident wave covers N, three weight rows per warp in a single
+  // batch (decode-sized launches, latency-bound); beyond that, two rows per warp
+  // with the next batch in flight, the fastest streaming shape measured (a
+  // 263 MB launch at M = 4: 2.98 TB/s, against 2.25 with three rows and 2.52
+  // with one)
+  if (MB <= 4 && N >= (int64_t)num_sms() * kGemvWarps * 3 * 3 / 2) {
+    if (N <= (int64_t)num_sms() * 2 * kGemvWarps * 3)
+      return launch_cfg<MB, 2, (MB <= 4 ? 3 : 1), false>(qa, asum, sa, w4, sw, y, M, N, K, s,
+                                                         pdl);
+    return launch_cfg<MB, 2, (MB <= 4 ? 2 : 1), true>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  }
   return launch_rpw<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
