@@ -926,8 +926,8 @@ lq_status lq_cta_create(const float* d_U, const float* d_V, int64_t d, int32_t r
       return LQ_ERR_ARG;
     }
   }
-  if (d % 32) {
-    set_error("CTA width d=%lld must be a multiple of 32", (long long)d);
+  if (d % 32 || d > 6144) {
+    set_error("CTA width d=%lld must be a multiple of 32 and at most 6144", (long long)d);
     return LQ_ERR_SHAPE;
   }
   lq_cta* c = new lq_cta();

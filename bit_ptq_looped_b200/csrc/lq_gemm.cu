@@ -619,22 +619,37 @@ __global__ void __launch_bounds__(H_THREADS, 1)
   }
 }
 
-// X (R x K bf16, row-major) -> Xt (K x Rp, zero columns past R)
-__global__ void k_transpose_bf16(const uint16_t* __restrict__ X, int64_t R, int64_t K,
-                                 int64_t Rp, uint16_t* __restrict__ Xt) {
-  __shared__ uint16_t tile[64][66];
+// X (R x K bf16, row-major) -> Xt (K x Rp, zero columns past R).  A block
+// moves a 64 x 64 tile with 16-byte loads and stores on both sides.
+__global__ void __launch_bounds__(256) k_transpose_bf16(const uint16_t* __restrict__ X,
+                                                        int64_t R, int64_t K, int64_t Rp,
+                                                        uint16_t* __restrict__ Xt) {
+  __shared__ uint16_t tile[64][64 + 2];
   pdl_trigger();
   const int64_t r0 = (int64_t)blockIdx.x * 64, k0 = (int64_t)blockIdx.y * 64;
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 256 threads: 64 x 4
-  for (int i = ty; i < 64; i += 4) {
-    const int64_t r = r0 + i, k = k0 + tx;
-    tile[i][tx] = (r < R && k < K) ? X[r * K + k] : (uint16_t)0;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {  // 64 rows x 8 chunks of 8 elements
+    const int i = u * 256 + threadIdx.x, row = i >> 3, c8 = (i & 7) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r0 + row < R) v = __ldg(reinterpret_cast<const uint4*>(X + (r0 + row) * K + k0 + c8));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      tile[row][c8 + 2 * e] = (uint16_t)(w[e] & 0xFFFFu);
+      tile[row][c8 + 2 * e + 1] = (uint16_t)(w[e] >> 16);
+    }
   }
   __syncthreads();
   pdl_wait();  // the previous kernel may still read Xt
-  for (int i = ty; i < 64; i += 4) {
-    const int64_t k = k0 + i, r = r0 + tx;
-    if (k < K && r < Rp) Xt[k * Rp + r] = tile[tx][i];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {  // 64 output rows (k) x 8 chunks of 8 (r)
+    const int i = u * 256 + threadIdx.x, kk = i >> 3, r8 = (i & 7) * 8;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      w[e] = (uint32_t)tile[r8 + 2 * e][kk] | ((uint32_t)tile[r8 + 2 * e + 1][kk] << 16);
+    if (r0 + r8 < Rp)
+      *reinterpret_cast<uint4*>(Xt + (k0 + kk) * Rp + r0 + r8) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -646,7 +661,7 @@ cudaError_t launch_trajectory_hessian(const uint16_t* X, int64_t R, int64_t K, u
                                       float* H, int accumulate, cudaStream_t s,
                                       const char** why) {
   const int64_t Rp = hessian_rows_padded(R);
-  dim3 tg((unsigned)((Rp + 63) / 64), (unsigned)((K + 63) / 64));
+  dim3 tg((unsigned)(Rp / 64), (unsigned)(K / 64));  // Rp and K are multiples of 64
   cudaError_t e = launch_kernel(k_transpose_bf16, tg, dim3(256), 0, s, false, X, R, K, Rp, Xt);
   if (e != cudaSuccess) return e;
   CUtensorMap mX;

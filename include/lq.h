@@ -251,7 +251,7 @@ lq_status lq_loop_stack_slt(const void* d_x, int32_t x_dtype, int64_t M,
  *   d_U, d_V  d x rank float32 row-major (device), 1 <= rank <= 8;
  *   d_a, d_b  n_trans x d float32 row-major (device): a_t, b_t of transition t
  *             (t -> t + 1);  h_eta[n_trans] (host, finite): the gates.
- * d must be a multiple of 32 (LQ_ERR_SHAPE).  Synchronous.  LQ_ERR_ARG on null
+ * d must be a multiple of 32 and at most 6144 (LQ_ERR_SHAPE).  Synchronous.  LQ_ERR_ARG on null
  * pointers or bad sizes, LQ_ERR_CUDA on a failed copy or allocation.  Release
  * with lq_cta_free.
  */
