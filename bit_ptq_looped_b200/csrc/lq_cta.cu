@@ -52,12 +52,24 @@ __global__ void __launch_bounds__(kCtaThreads) k_cta_apply(
   const int d4 = d >> 2;
   for (int64_t r0 = (int64_t)blockIdx.x * 8; r0 < M; r0 += (int64_t)gridDim.x * 8) {
     const int nr = M - r0 < 8 ? (int)(M - r0) : 8;
-    // ---- the block's rows to shared memory (zeros past the last row)
-    for (int i = threadIdx.x; i < 8 * d4; i += kCtaThreads) {
-      const int rr = i / d4, c4 = i - rr * d4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (rr < nr) v = *reinterpret_cast<const float4*>(h + (r0 + rr) * (int64_t)d + 4 * c4);
-      *reinterpret_cast<float4*>(hs + rr * ld + 4 * c4) = v;
+    // ---- the block's rows to shared memory (zeros past the last row), four
+    // 16-byte loads of each thread in flight at a time
+    for (int base = 0; base < 8 * d4; base += 4 * kCtaThreads) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * kCtaThreads + threadIdx.x;
+        const int rr = i / d4, c4 = i - rr * d4;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < 8 * d4 && rr < nr)
+          v[u] = *reinterpret_cast<const float4*>(h + (r0 + rr) * (int64_t)d + 4 * c4);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * kCtaThreads + threadIdx.x;
+        const int rr = i / d4, c4 = i - rr * d4;
+        if (i < 8 * d4) *reinterpret_cast<float4*>(hs + rr * ld + 4 * c4) = v[u];
+      }
     }
     __syncthreads();
     // ---- pass 1: this warp's slice of p = h V

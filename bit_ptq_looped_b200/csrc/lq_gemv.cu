@@ -41,12 +41,13 @@ __device__ __forceinline__ int dp4a_us(uint32_t a_unsigned, uint32_t b_signed, i
 // RPW: weight rows per warp per batch; kDB: prefetch batch b + 1 while folding b
 // (worth its registers only when a warp has more than one batch).
 // shared layout: act vectors [(m * 2 + h) * G + g] (uint4), then asum[M * G], ssa[M * G].
-// (launch bounds: the streaming variant states a minimum of one block per SM so
-// that it keeps its prefetch registers, which measured faster than trading them
-// for occupancy; the single-batch decode variant keeps the occupancy that lets
-// the next kernels of a sequence start beside it)
+// (launch bounds: the streaming variant for up to 4 rows states a minimum of
+// one block per SM so that it keeps its prefetch registers, which measured
+// faster than trading them for occupancy; with 16 rows two blocks per SM
+// measured faster; the single-batch decode variant keeps the occupancy that
+// lets the next kernels of a sequence start beside it)
 template <int MB, int GPL, int RPW, bool kDB>
-__global__ void __launch_bounds__(kGemvThreads, kDB ? 1 : 3) k_group_gemv(
+__global__ void __launch_bounds__(kGemvThreads, kDB ? (MB >= 16 ? 2 : 1) : 3) k_group_gemv(
     const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
     const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
     int N, int K) {
