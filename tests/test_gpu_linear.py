@@ -89,11 +89,12 @@ def test_loop_linear_decode(M, N, a_bits):
         linear_parity(host(y), x, ol, t, host(q8), host(s), layer.w_flips)
 
 
-@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("M", [1, 4, 6, 9, 16])
 def test_gemv_many_row_batches(M):
     """N = 3 * 5632 + 8 weight rows: more rows than one resident wave of warps
     holds, so every warp folds several batches through both register sets of
-    the weight prefetch, and the last batch is ragged."""
+    the weight prefetch, and the last batch is ragged; 6, 9 and 16 tokens take
+    the tensor-core GEMV (one and two blocks of 8 tokens, partly empty)."""
     N = 3 * 5632 + 8
     wl = synth.Workload(f"decode_M{M}_N{N}", M=M, T=1,
                         linears=(synth.Linear("dec", 2048, N, 32, 64, 0),), a_bits=8,
