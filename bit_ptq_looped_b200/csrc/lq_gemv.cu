@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_group_gemv_mma(
 }
 
 size_t gemv_smem_bytes(int64_t M, int64_t G) { return (size_t)M * G * (32 + 8); }
+constexpr size_t kGemvMaxSmem = 200u * 1024u;  // the activation bound of the GEMV path
 
 template <int MB, int GPL, int RPW, bool kDB>
 cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
@@ -330,10 +331,14 @@ cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const
     std::lock_guard<std::mutex> lk(mu);
     auto it = per_sm_cache.find(smem);
     if (it == per_sm_cache.end()) {
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)std::max<size_t>(smem, 1));
-      if (e != cudaSuccess) return e;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemvThreads, smem);
+      // the attribute is one per function: raise it once to the largest activation
+      // any call can stage, never lower it under an earlier call's size
+      if (per_sm_cache.empty()) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kGemvMaxSmem);
+        if (e != cudaSuccess) return e;
+      }
+      cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemvThreads, smem);
       if (e != cudaSuccess) return e;
       if (per_sm < 1) return cudaErrorInvalidConfiguration;
       per_sm_cache.emplace(smem, per_sm);
@@ -373,10 +378,14 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
     std::lock_guard<std::mutex> lk(mu);
     auto it = per_sm_cache.find(smem);
     if (it == per_sm_cache.end()) {
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)std::max<size_t>(smem, 1));
-      if (e != cudaSuccess) return e;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemvThreads, smem);
+      // the attribute is one per function: raise it once to the largest activation
+      // any call can stage, never lower it under an earlier call's size
+      if (per_sm_cache.empty()) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kGemvMaxSmem);
+        if (e != cudaSuccess) return e;
+      }
+      cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemvThreads, smem);
       if (e != cudaSuccess) return e;
       if (per_sm < 1) return cudaErrorInvalidConfiguration;
       per_sm_cache.emplace(smem, per_sm);
@@ -417,7 +426,9 @@ cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa
                               const uint8_t* w4, const float* sw, float* y, int64_t M, int64_t N,
                               int64_t K, cudaStream_t s, bool pdl) {
   if (M == 0 || N == 0) return cudaSuccess;
-  if (K > (int64_t)kGroup * 32 * 8 || M > kGemvMaxM) return cudaErrorInvalidValue;
+  if (K > (int64_t)kGroup * 32 * 8 || M > kGemvMaxM ||
+      gemv_smem_bytes(M, K / kGroup) > kGemvMaxSmem)
+    return cudaErrorInvalidValue;
   if (M <= 1) return launch_mb<1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
   if (M <= 4) return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
   // 5 to 16 tokens: integer tensor-core MMAs (8 tokens per MMA)

@@ -19,6 +19,8 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
 
 #include "lq_common.cuh"
 
@@ -723,8 +725,19 @@ __global__ void k_transpose_f32(const float* __restrict__ in, int64_t rows, int6
 
 template <typename F>
 cudaError_t set_smem(F* f, size_t bytes) {
-  static_assert(sizeof(F*) > 0, "");
-  return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  // The limit is one per function and recorded schedules (CUDA graphs) launch
+  // with whatever it is at replay: only ever raise it, so that a smaller call
+  // never lowers it under a larger one recorded earlier.
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, size_t> raised;  // per device and function
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  size_t& cur = raised[{dev, (const void*)f}];
+  if (bytes <= cur) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) cur = bytes;
+  return e;
 }
 
 }  // namespace
