@@ -4,8 +4,10 @@
 //
 // Same arithmetic as the tensor-core GEMM, for the decode regime where each
 // loop reads the packed 4-bit weights once and the activation is a handful of
-// rows.  Up to 4 tokens use dp4a on the CUDA cores (below); 5 to 16 tokens use
-// the integer tensor-core MMA (k_group_gemv_mma, further down).
+// rows.  One token, and 2 to 4 tokens on launches of less than about one
+// resident wave of rows, use dp4a on the CUDA cores (below); 5 to 16 tokens,
+// and 2 to 4 on streaming launches, use the integer tensor-core MMA
+// (k_group_gemv_mma, further down).
 // Warp w of the grid owns weight rows w, w + W, w + 2W, ... (W warps in
 // the grid); lane L owns groups L, L + 32, ... of each row: one 16-byte load
 // brings the 32 packed codes of a group, one 4-byte load its step.  The
@@ -23,6 +25,7 @@
 // overlaps the quantizer that produces its activation.
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 #include <unordered_map>
 
 #include "lq_common.cuh"
@@ -185,137 +188,248 @@ __global__ void __launch_bounds__(kGemvThreads, kDB ? 1 : 3) k_group_gemv(
 }
 
 // ---------------------------------------------------------------------------
-// 5 to 16 tokens: the integer dots on the tensor cores (mma.sync m16n8k32,
-// u8 x s8 -> s32).  A warp takes 16 weight rows at a time and walks all groups
-// of K; one MMA per group and block of 8 tokens.  The group's 32 codes form
-// the MMA's K dimension in the order of the packed words: thread (g, t) of the
-// MMA holds k-quad t = the low nibbles of weight word t (codes 8t, 8t+2, 8t+4,
-// 8t+6) and k-quad t + 4 = its high nibbles, and the activation fragments are
-// the matching even and odd code words e_t, o_t of the kOpGemvAct layout.
-// Weight nibbles enter as v ^ 8 = q_w + 8 (unsigned); the accumulator starts at
-// -8 * sum q_a, so the MMA returns sum q_w q_a exactly.  Each output (row,
-// token) belongs to one thread, which folds s_w * s_a * sum per group.
+// 2 to 16 tokens on a streaming launch, and 5 to 16 tokens always: the integer
+// dots on the tensor cores (mma.sync m16n8k32, u8 x s8 -> s32), one MMA per
+// group, 16 weight rows and block of 8 tokens.
+//
+// Fragments.  The group's 32 codes form the MMA's K dimension in the order of
+// the packed words: thread (g, t) of the MMA holds k-quad t = the low nibbles
+// of weight word t (codes 8t, 8t+2, 8t+4, 8t+6) and k-quad t + 4 = its high
+// nibbles; the activation fragments are the matching even and odd code words
+// e_t, o_t of the kOpGemvAct layout.  Weight nibbles enter as v ^ 8 = q_w + 8
+// (unsigned), and the MMA adds sum (q_w + 8) q_a to a constant accumulator
+// input of 1.5 * 2^23 (as an integer): its result is the float bit pattern of
+// 1.5 * 2^23 + sum (q_w + 8) q_a (|sum| < 2^22), and one float add of
+// -(1.5 * 2^23 + 8 sum q_a) (exact: integers below 2^24) leaves the exact
+// dot sum q_w q_a, with no int-to-float conversion.  Each output (row, token)
+// belongs to one thread, which folds s_w * s_a * dot per group in float32
+// (packed f32x2 arithmetic).
+//
+// Weight stream.  Each warp owns a ring of kS shared-memory stages; a stage is
+// 16 rows x kU groups of packed codes (16 bytes per row and group) plus their
+// steps, brought in by cp.async (the 8 lanes of a row copy 128 contiguous
+// bytes) and read back with ldmatrix, which hands thread (g, t) word t of row
+// g: the A fragment, transposed in the load.  Chunks are stored XOR-swizzled
+// by row so that the 8 row addresses of an ldmatrix hit distinct banks.  The
+// warp walks its row blocks (rb = warp, + all warps, ...) stage by stage with
+// kS - 1 stages in flight; cp.async.wait_group is the only wait.
+// The activation (codes of all tokens) is staged once per block in shared
+// memory in MMA-fragment order (lane-contiguous, conflict-free), with the
+// float offsets -(1.5 * 2^23 + 8 sum q_a) and s_a of each (group, token block,
+// thread) in one 16-byte record.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void mma_u8s8_16832(int (&c)[4], uint32_t a0, uint32_t a1,
+// d = A B + c (every accumulator input c)
+__device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+                                               uint32_t b1, int c) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%11,%12,%13};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c), "r"(c), "r"(c), "r"(c));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
-template <int NB>  // blocks of 8 tokens
-__global__ void __launch_bounds__(kGemvThreads, 2) k_group_gemv_mma(
+constexpr int kMmaWarps = 8;
+constexpr int kFloatBias = 0x4B400000;  // bit pattern of 1.5 * 2^23 = 12582912
+
+// shared memory of one block: activation fragments, then kMmaWarps rings
+__host__ __device__ constexpr size_t mma_act_bytes(int NB, int64_t G) {
+  return (size_t)G * NB * (32 * 8 + 4 * 16);  // uint2 [G][NB][32], float4 [G][NB][4]
+}
+__host__ __device__ constexpr size_t mma_stage_bytes(int kU) { return (size_t)16 * kU * (16 + 4); }
+
+template <int NB, int kS, int kU, int kMinBlocks>
+__global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
     const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
     const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
     int N, int K) {
+  static_assert(kU % 8 == 0 && kS >= 2, "stages of whole 8-chunk swizzle blocks, double buffered");
+  constexpr int kStageW = 16 * kU * 16;  // packed codes of a stage
+  constexpr int kStage = (int)mma_stage_bytes(kU);
   extern __shared__ __align__(16) unsigned char smem_raw[];
   pdl_trigger();
   const int G = K / kGroup;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int gw = blockIdx.x * kGemvWarps + warp, W = gridDim.x * kGemvWarps;
+  const int gw = blockIdx.x * kMmaWarps + warp, W = gridDim.x * kMmaWarps;
   const size_t rowstride = (size_t)K / 2;
+  unsigned char* ring = smem_raw + mma_act_bytes(NB, G) + (size_t)warp * kS * kStage;
+  const uint32_t ring_s = smem_u32(ring);
+  const int stages_per_rb = (G + kU - 1) / kU;
+  const int n_rb = (N + 15) / 16;
+  const int my_rb = gw < n_rb ? (n_rb - gw + W - 1) / W : 0;
+  const int n_stages = my_rb * stages_per_rb;
+  const bool vec_steps = (G & 3) == 0;  // 16-byte step chunks are aligned
 
-  // first weight words of this warp's first row block, before the wait
-  constexpr int kU = 4;  // groups per load batch
-  uint32_t wA[kU], wB[kU];
-  float swA[kU], swB[kU];
-  auto load_groups = [&](int n0, int g0) {
-    const int na = n0 + g, nb = n0 + g + 8;
+  // copy stage b of this warp (row block gw + (b / stages_per_rb) * W, groups
+  // (b % stages_per_rb) * kU ..) into slot b % kS; one commit group per stage
+  auto issue = [&](int b) {
+    if (b < n_stages) {
+      const int rb = gw + (b / stages_per_rb) * W, g0 = (b % stages_per_rb) * kU;
+      const uint32_t st = ring_s + (uint32_t)((b % kS) * kStage);
+      const bool full = rb * 16 + 16 <= N && g0 + kU <= G;  // no row or group outside
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int grp = g0 + u;
-      const bool oka = na < N && grp < G, okb = nb < N && grp < G;
-      wA[u] = oka ? __ldg(reinterpret_cast<const uint32_t*>(w4 + (size_t)na * rowstride) +
-                          grp * 4 + t)
-                  : 0x88888888u;
-      wB[u] = okb ? __ldg(reinterpret_cast<const uint32_t*>(w4 + (size_t)nb * rowstride) +
-                          grp * 4 + t)
-                  : 0x88888888u;
-      swA[u] = oka ? __ldg(sw + (size_t)na * G + grp) : 0.f;
-      swB[u] = okb ? __ldg(sw + (size_t)nb * G + grp) : 0.f;
+      for (int i = 0; i < kU / 2; ++i) {
+        const int c = lane + 32 * i, r = c / kU, u = c % kU;
+        const int n = rb * 16 + r, grp = g0 + u;
+        if (full || (n < N && grp < G))
+          cp_async16(st + (uint32_t)((r * kU + (u ^ (r & 7))) * 16),
+                     w4 + (size_t)n * rowstride + (size_t)grp * 16);
+      }
+#pragma unroll
+      for (int i = 0; i < kU / 8; ++i) {
+        const int c = lane + 32 * i, r = c / (kU / 4), h = c % (kU / 4), n = rb * 16 + r;
+        const int grp = g0 + 4 * h;
+        const uint32_t dst = st + kStageW + (uint32_t)(r * kU * 4 + h * 16);
+        if (vec_steps) {
+          if (n < N && grp < G) cp_async16(dst, sw + (size_t)n * G + grp);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (n < N && grp + e < G) cp_async4(dst + 4 * e, sw + (size_t)n * G + grp + e);
+        }
+      }
     }
+    cp_async_commit();
   };
-  if (gw * 16 < N) load_groups(gw * 16, 0);
+  // the weight stream does not depend on the previous kernel: start it first
+#pragma unroll
+  for (int b = 0; b < kS - 1; ++b) issue(b);
 
   pdl_wait();  // the activation is the previous kernel's output
-  uint4* act = reinterpret_cast<uint4*>(smem_raw);
-  int* asum = reinterpret_cast<int*>(act + (size_t)M * 2 * G);
-  float* ssa = reinterpret_cast<float*>(asum + (size_t)M * G);
+  uint2* bfrag = reinterpret_cast<uint2*>(smem_raw);
+  float4* offs_sa = reinterpret_cast<float4*>(bfrag + (size_t)G * NB * 32);
   {
-    const int n_vec = M * 2 * G;
-    const uint4* src = reinterpret_cast<const uint4*>(qa);
-    for (int i = threadIdx.x; i < n_vec; i += kGemvThreads) act[i] = __ldg(src + i);
-    for (int i = threadIdx.x; i < M * G; i += kGemvThreads) {
-      asum[i] = __ldg(asum_g + i);
-      ssa[i] = __ldg(sa + i);
+    // activation words in source order: uint2 ((m * 2 + h) * G + grp) * 2 + c2 is
+    // the fragment of lane (m % 8) * 4 + 2h + c2 in token block m / 8
+    const uint2* src = reinterpret_cast<const uint2*>(qa);
+    const int n_src = M * 2 * G * 2;
+    for (int i = threadIdx.x; i < n_src; i += kMmaWarps * 32) {
+      const int c2 = i & 1, grp = (i >> 1) % G, mh = (i >> 1) / G, h = mh & 1, m = mh >> 1;
+      bfrag[((size_t)grp * NB + (m >> 3)) * 32 + (m & 7) * 4 + 2 * h + c2] = __ldg(src + i);
+    }
+    const int n_pad = (NB * 8 - M) * 2 * G * 2;  // empty token slots: zero codes
+    for (int i = threadIdx.x; i < n_pad; i += kMmaWarps * 32) {
+      const int c2 = i & 1, grp = (i >> 1) % G, mh = (i >> 1) / G, h = mh & 1, m = M + (mh >> 1);
+      bfrag[((size_t)grp * NB + (m >> 3)) * 32 + (m & 7) * 4 + 2 * h + c2] = make_uint2(0u, 0u);
+    }
+    for (int i = threadIdx.x; i < G * NB * 4; i += kMmaWarps * 32) {
+      const int tt = i & 3, j = (i >> 2) % NB, grp = (i >> 2) / NB;
+      const int m0 = j * 8 + 2 * tt;
+      const float o0 = m0 < M ? 8.f * (float)__ldg(asum_g + (size_t)m0 * G + grp) : 0.f;
+      const float o1 = m0 + 1 < M ? 8.f * (float)__ldg(asum_g + (size_t)(m0 + 1) * G + grp) : 0.f;
+      offs_sa[i] = make_float4(-12582912.0f - o0, -12582912.0f - o1,
+                               m0 < M ? __ldg(sa + (size_t)m0 * G + grp) : 0.f,
+                               m0 + 1 < M ? __ldg(sa + (size_t)(m0 + 1) * G + grp) : 0.f);
     }
   }
   __syncthreads();
-  const uint32_t* act32 = reinterpret_cast<const uint32_t*>(act);
 
-  for (int rb = gw; rb * 16 < N; rb += W) {
-    const int n0 = rb * 16;
-    float acc[NB][4];
+  float2 acc[NB][2];  // [token block][row g, row g + 8] x (token m0, m0 + 1)
 #pragma unroll
-    for (int j = 0; j < NB; ++j)
+  for (int j = 0; j < NB; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
+  // group pair (u, u + 1) of a stage: ldmatrix matrices 0-3 = rows 0-7 / 8-15 of
+  // group u, then of u + 1; lane L addresses row L % 8 of matrix L / 8
+  const int lm_row = (lane & 7) + 8 * ((lane >> 3) & 1), lm_du = lane >> 4;
+  auto fold_group = [&](int grp, uint32_t wa, uint32_t wb, float swa, float swb) {
+    const uint32_t xa = wa ^ 0x88888888u, xb = wb ^ 0x88888888u;
+    const uint32_t a0 = xa & 0x0F0F0F0Fu, a1 = xb & 0x0F0F0F0Fu;
+    const uint32_t a2 = (xa >> 4) & 0x0F0F0F0Fu, a3 = (xb >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-    for (int g0 = 0; g0 < G; g0 += kU) {
-      if (rb != gw || g0 != 0) load_groups(n0, g0);
+    for (int j = 0; j < NB; ++j) {
+      const size_t f = (size_t)grp * NB + j;
+      const uint2 b = bfrag[f * 32 + lane];
+      const float4 os = offs_sa[f * 4 + t];
+      const float2 off = make_float2(os.x, os.y), s01 = make_float2(os.z, os.w);
+      int d[4];
+      mma_u8s8_16832(d, a0, a1, a2, a3, b.x, b.y, kFloatBias);
+      const float2 da = fadd2(make_float2(__int_as_float(d[0]), __int_as_float(d[1])), off);
+      const float2 db = fadd2(make_float2(__int_as_float(d[2]), __int_as_float(d[3])), off);
+      acc[j][0] = ffma2(fmul2(make_float2(swa, swa), s01), da, acc[j][0]);
+      acc[j][1] = ffma2(fmul2(make_float2(swb, swb), s01), db, acc[j][1]);
+    }
+  };
+  // the groups of one stage; kFull: all kU groups exist (no per-group branches,
+  // so that the loads and MMAs of the whole stage can be scheduled together)
+  auto fold_stage = [&](auto full_tag, uint32_t st, const float* ssw, int g0) {
+    constexpr bool kFull = decltype(full_tag)::value;
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int grp = g0 + u;
-        if (grp < G) {
-          const uint32_t xa = wA[u] ^ 0x88888888u, xb = wB[u] ^ 0x88888888u;
-          const uint32_t a0 = xa & 0x0F0F0F0Fu, a1 = xb & 0x0F0F0F0Fu;
-          const uint32_t a2 = (xa >> 4) & 0x0F0F0F0Fu, a3 = (xb >> 4) & 0x0F0F0F0Fu;
+    for (int q = 0; q < kU / 4; ++q) {
+      if (kFull || g0 + 4 * q < G) {
+        const float4 fa = *reinterpret_cast<const float4*>(ssw + g * kU + 4 * q);
+        const float4 fb = *reinterpret_cast<const float4*>(ssw + (g + 8) * kU + 4 * q);
+        const float fa4[4] = {fa.x, fa.y, fa.z, fa.w}, fb4[4] = {fb.x, fb.y, fb.z, fb.w};
 #pragma unroll
-          for (int j = 0; j < NB; ++j) {
-            const int mb = j * 8 + g;          // token of the B fragment column
-            const int m0 = j * 8 + 2 * t;      // tokens of this thread's C columns
-            uint32_t b0 = 0, b1 = 0;
-            if (mb < M) {
-              const uint32_t* e = act32 + ((size_t)(mb * 2 + (t >> 1)) * G + grp) * 4 + (t & 1) * 2;
-              b0 = e[0];
-              b1 = e[1];
-            }
-            const bool v0 = m0 < M, v1 = m0 + 1 < M;
-            const int c0 = v0 ? -8 * asum[m0 * G + grp] : 0;
-            const int c1 = v1 ? -8 * asum[(m0 + 1) * G + grp] : 0;
-            int c[4] = {c0, c1, c0, c1};
-            mma_u8s8_16832(c, a0, a1, a2, a3, b0, b1);
-            const float s0 = v0 ? ssa[m0 * G + grp] : 0.f;
-            const float s1 = v1 ? ssa[(m0 + 1) * G + grp] : 0.f;
-            acc[j][0] = fmaf(swA[u] * s0, (float)c[0], acc[j][0]);
-            acc[j][1] = fmaf(swA[u] * s1, (float)c[1], acc[j][1]);
-            acc[j][2] = fmaf(swB[u] * s0, (float)c[2], acc[j][2]);
-            acc[j][3] = fmaf(swB[u] * s1, (float)c[3], acc[j][3]);
+        for (int p = 0; p < 2; ++p) {
+          const int u = 4 * q + 2 * p;
+          if (kFull || g0 + u < G) {
+            uint32_t w[4];
+            const int uu = u + lm_du;
+            ldmatrix_x4(st + (uint32_t)((lm_row * kU + (uu ^ (lm_row & 7))) * 16), w);
+            fold_group(g0 + u, w[0], w[1], fa4[2 * p], fb4[2 * p]);
+            if (kFull || g0 + u + 1 < G) fold_group(g0 + u + 1, w[2], w[3], fa4[2 * p + 1], fb4[2 * p + 1]);
           }
         }
       }
     }
-    const int na = n0 + g, nb = n0 + g + 8;
+  };
+
+  int rb = gw, g0 = 0;
+  for (int b = 0; b < n_stages; ++b) {
+    issue(b + kS - 1);
+    cp_async_wait<kS - 1>();  // this thread's copies of stage b have landed
+    __syncwarp();             // ... and every other lane's
+    const uint32_t st = ring_s + (uint32_t)((b % kS) * kStage);
+    const float* ssw = reinterpret_cast<const float*>(ring + (b % kS) * kStage + kStageW);
+    if (g0 + kU <= G)
+      fold_stage(std::true_type{}, st, ssw, g0);
+    else
+      fold_stage(std::false_type{}, st, ssw, g0);
+    __syncwarp();  // every lane is done with this slot before it is refilled
+    if (g0 + kU >= G) {  // last stage of the row block: write its outputs
+      const int na = rb * 16 + g, nb = na + 8;
 #pragma unroll
-    for (int j = 0; j < NB; ++j) {
-      const int m0 = j * 8 + 2 * t;
-      if (na < N) {
-        if (m0 < M) y[(size_t)m0 * N + na] = acc[j][0];
-        if (m0 + 1 < M) y[(size_t)(m0 + 1) * N + na] = acc[j][1];
+      for (int j = 0; j < NB; ++j) {
+        const int m0 = j * 8 + 2 * t;
+        if (na < N) {
+          if (m0 < M) y[(size_t)m0 * N + na] = acc[j][0].x;
+          if (m0 + 1 < M) y[(size_t)(m0 + 1) * N + na] = acc[j][0].y;
+        }
+        if (nb < N) {
+          if (m0 < M) y[(size_t)m0 * N + nb] = acc[j][1].x;
+          if (m0 + 1 < M) y[(size_t)(m0 + 1) * N + nb] = acc[j][1].y;
+        }
+        acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
       }
-      if (nb < N) {
-        if (m0 < M) y[(size_t)m0 * N + nb] = acc[j][2];
-        if (m0 + 1 < M) y[(size_t)(m0 + 1) * N + nb] = acc[j][3];
-      }
+      g0 = 0;
+      rb += W;
+    } else {
+      g0 += kU;
     }
   }
+  cp_async_wait<0>();  // no copy outlives the block
 }
 
 size_t gemv_smem_bytes(int64_t M, int64_t G) { return (size_t)M * G * (32 + 8); }
 constexpr size_t kGemvMaxSmem = 200u * 1024u;  // the activation bound of the GEMV path
+constexpr size_t kMmaMaxSmem = 227u * 1024u;   // opt-in shared memory of one block
 
 template <int MB, int GPL, int RPW, bool kDB>
 cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
@@ -365,12 +479,14 @@ cudaError_t launch_rpw(const int8_t* qa, const int* asum, const float* sa, const
   return launch_cfg<MB, GPL, RPW, true>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
-template <int NB>
+template <int NB, int kS, int kU>
 cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                        const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
                        bool pdl) {
-  const size_t smem = gemv_smem_bytes(M, K / kGroup);
-  auto* k = k_group_gemv_mma<NB>;
+  const int64_t G = K / kGroup;
+  const size_t smem = mma_act_bytes(NB, G) + (size_t)kMmaWarps * kS * mma_stage_bytes(kU);
+  if (smem > kMmaMaxSmem) return cudaErrorInvalidValue;
+  auto* k = k_group_gemv_mma<NB, kS, kU, 2>;
   static std::mutex mu;
   static std::unordered_map<size_t, int> per_sm_cache;
   int per_sm = 0;
@@ -378,14 +494,14 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
     std::lock_guard<std::mutex> lk(mu);
     auto it = per_sm_cache.find(smem);
     if (it == per_sm_cache.end()) {
-      // the attribute is one per function: raise it once to the largest activation
-      // any call can stage, never lower it under an earlier call's size
+      // one attribute per function: raised once to the largest size any call uses
       if (per_sm_cache.empty()) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kGemvMaxSmem);
+                                             (int)kMmaMaxSmem);
         if (e != cudaSuccess) return e;
       }
-      cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemvThreads, smem);
+      cudaError_t e =
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kMmaWarps * 32, smem);
       if (e != cudaSuccess) return e;
       if (per_sm < 1) return cudaErrorInvalidConfiguration;
       per_sm_cache.emplace(smem, per_sm);
@@ -393,11 +509,24 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
       per_sm = it->second;
     }
   }
-  const int64_t warps_needed = (N + 15) / 16;
-  const int64_t want = (warps_needed + kGemvWarps - 1) / kGemvWarps;
+  const int64_t row_blocks = (N + 15) / 16;
+  const int64_t want = (row_blocks + kMmaWarps - 1) / kMmaWarps;
   const int64_t blocks = std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
-  return launch_kernel(k, dim3((unsigned)blocks), dim3(kGemvThreads), smem, s, pdl, qa, asum, sa,
-                       w4, sw, y, (int)M, (int)N, (int)K);
+  return launch_kernel(k, dim3((unsigned)blocks), dim3(kMmaWarps * 32), smem, s, pdl, qa, asum,
+                       sa, w4, sw, y, (int)M, (int)N, (int)K);
+}
+
+// the tensor-core GEMV for M tokens: one block of 8 tokens with 16-group
+// stages (2 in flight per warp), or two blocks with 8-group stages (3, or 2
+// when the activation leaves too little shared memory for 3)
+cudaError_t launch_tc(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
+                      const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                      bool pdl) {
+  const int64_t G = K / kGroup;
+  if (M <= 8) return launch_mma<1, 2, 16>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  if (mma_act_bytes(2, G) + (size_t)kMmaWarps * 3 * mma_stage_bytes(8) <= kMmaMaxSmem)
+    return launch_mma<2, 3, 8>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_mma<2, 2, 8>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
 template <int MB>
@@ -429,11 +558,18 @@ cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa
   if (K > (int64_t)kGroup * 32 * 8 || M > kGemvMaxM ||
       gemv_smem_bytes(M, K / kGroup) > kGemvMaxSmem)
     return cudaErrorInvalidValue;
+  // one token: dp4a (a 263 MB launch timed alone: 5.47 TB/s, against 5.25
+  // on the tensor-core path, whose block prologue shows when launches are
+  // isolated)
   if (M <= 1) return launch_mb<1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  if (M <= 4) return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  // 5 to 16 tokens: integer tensor-core MMAs (8 tokens per MMA)
-  if (M <= 8) return launch_mma<1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  return launch_mma<2>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  // 2 to 4 tokens: dp4a while the rows fit in about one resident wave of
+  // warps (one memory latency per warp, the decode-sized launches); once the
+  // launch streams at least a wave of 16-row blocks, the tensor-core path
+  // with its deeper weight pipeline (a 263 MB launch at M = 4: 5.3 TB/s
+  // against 2.9 with dp4a)
+  if (M <= 4 && N < (int64_t)num_sms() * 2 * kMmaWarps * 16)
+    return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_tc(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
 }  // namespace lq

@@ -89,26 +89,56 @@ def test_loop_linear_decode(M, N, a_bits):
         linear_parity(host(y), x, ol, t, host(q8), host(s), layer.w_flips)
 
 
+def _gemv_case(M, N, K, a, b, a_bits, t=0):
+    """One decode-sized linear (M tokens, K = a * b, N weight rows) through the
+    library against the oracle."""
+    wl = synth.Workload(f"decode_M{M}_N{N}_K{K}", M=M, T=t + 1,
+                        linears=(synth.Linear("dec", K, N, a, b, 0),), a_bits=a_bits,
+                        outlier_frac=0.02, outlier_mult=20.0, x_dtype="bf16",
+                        description="decode GEMV case")
+    (mp,) = synth.module_params(wl)
+    (lin,) = wl.linears
+    layer, ol = make_layer(mp, a_bits)
+    x = synth.loop_input(wl, lin, t)
+    xd = act_tensor(x, wl.x_dtype)
+    y = lq.lq_loop_linear(xd, layer, t)
+    q8, _, s = lq.lq_quantize_act(xd, dev(mp.P1), dev(mp.P2), float(mp.las[t]), a_bits)
+    torch.cuda.synchronize()
+    linear_parity(host(y), x, ol, t, host(q8), host(s), layer.w_flips)
+
+
 @pytest.mark.parametrize("M", [1, 4, 6, 9, 16])
 def test_gemv_many_row_batches(M):
     """N = 3 * 5632 + 8 weight rows: more rows than one resident wave of warps
-    holds, so every warp folds several batches through both register sets of
-    the weight prefetch, and the last batch is ragged; 6, 9 and 16 tokens take
-    the tensor-core GEMV (one and two blocks of 8 tokens, partly empty)."""
-    N = 3 * 5632 + 8
-    wl = synth.Workload(f"decode_M{M}_N{N}", M=M, T=1,
-                        linears=(synth.Linear("dec", 2048, N, 32, 64, 0),), a_bits=8,
-                        outlier_frac=0.02, outlier_mult=20.0, x_dtype="bf16",
-                        description="decode GEMV with several row batches per warp")
-    (mp,) = synth.module_params(wl)
-    (lin,) = wl.linears
-    layer, ol = make_layer(mp, 8)
-    x = synth.loop_input(wl, lin, 0)
-    xd = act_tensor(x, wl.x_dtype)
-    y = lq.lq_loop_linear(xd, layer, 0)
-    q8, _, s = lq.lq_quantize_act(xd, dev(mp.P1), dev(mp.P2), float(mp.las[0]), 8)
-    torch.cuda.synchronize()
-    linear_parity(host(y), x, ol, 0, host(q8), host(s), layer.w_flips)
+    holds, so every warp folds several batches (dp4a) or several row blocks
+    through its stage ring (tensor-core path, 6, 9 and 16 tokens: one and two
+    blocks of 8 tokens, partly empty), and the last rows are ragged."""
+    _gemv_case(M, 3 * 5632 + 8, 2048, 32, 64, 8)
+
+
+@pytest.mark.parametrize("M,a_bits", [(1, 8), (2, 8), (3, 4), (4, 8), (4, 4)])
+def test_gemv_streaming_few_tokens(M, a_bits):
+    """A launch of more than one wave of 16-row blocks (N = 148 x 256 + 8
+    rows): 2 to 4 tokens take the tensor-core path with its stage ring, one
+    token the dp4a path with two weight-row batches in flight per warp; the
+    last rows are ragged."""
+    _gemv_case(M, 148 * 256 + 8, 2048, 32, 64, a_bits)
+
+
+@pytest.mark.parametrize("K,a,b", [(128, 16, 8), (384, 16, 24), (1152, 16, 72), (5632, 64, 88)])
+@pytest.mark.parametrize("M", [5, 16])
+def test_gemv_tensor_core_group_tails(K, a, b, M):
+    """Group counts against the stages of 16 (up to 8 tokens) and 8 groups
+    (9 to 16 tokens): G = 4 (fewer groups than a stage), 12 and 36 (a partial
+    last stage), 176 (whole stages); N = 1000 rows (a ragged row block)."""
+    _gemv_case(M, 1000, K, a, b, 8)
+
+
+def test_gemv_tensor_core_large_k():
+    """K = 7680 = 96 x 80 at 16 tokens, the largest Kronecker shape the
+    rotation stages: the activation fragments (150 KB) and three stages per
+    warp fill 210 KB of shared memory."""
+    _gemv_case(16, 520, 7680, 96, 80, 4)
 
 
 @pytest.mark.parametrize("M", [0, 1, 17, 129, 300])
