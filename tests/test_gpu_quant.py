@@ -173,3 +173,49 @@ def test_fold_weights(ab):
     lhs = x @ W.astype(np.float64).T
     rhs = (x @ np.kron(P1.astype(np.float64), P2.astype(np.float64))) @ got.astype(np.float64).T
     assert np.max(np.abs(lhs - rhs)) <= 1e-5 * np.max(np.abs(lhs))
+
+
+def test_hand_examples_through_the_kernels():
+    """The hand-derived cases of tests/golden/qa_hand_examples.json (worked out
+    from Section 2 Eq. (4) of the LoopQ specification under the readings stated
+    there) through the CUDA quantizer and weight packer, bit for bit: steps,
+    codes (the exact ties included, one of which separates a true division from
+    a reciprocal multiply) and packed bytes."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "qa_hand_examples.json")) as f:
+        gold = json.load(f)
+    for case in gold["activation_cases"]:
+        x = np.zeros((1, 32), np.float32)
+        x[0, :len(case["x"])] = case["x"]
+        q8, q4, s = lq.lq_quantize_act(dev(x), None, None, case["c"], case["bits"],
+                                       want_codes4=case["bits"] == 4)
+        torch.cuda.synchronize()
+        n = len(case["codes"])
+        if "scale" in case:
+            want_s = np.float32(case["scale"])
+        else:  # s = fl32(fl32(c * absmax) / q_max), as the case's note works it out
+            qmax = 7 if case["bits"] == 4 else 127
+            want_s = np.float32(np.float32(case["c"]) * np.float32(np.abs(case["x"]).max())) \
+                / np.float32(qmax)
+        assert host(s)[0, 0] == want_s, case["name"]
+        assert list(host(q8)[0, :n]) == case["codes"], case["name"]
+        assert not host(q8)[0, n:].any(), case["name"]
+        if case["bits"] == 4:
+            assert np.array_equal(host(q4)[0], O.pack_int4(host(q8))[0]), case["name"]
+    for case in gold["weight_cases"]:
+        w = np.zeros((1, 32), np.float32)
+        w[0, :len(case["w"])] = case["w"]
+        c4, sc = lq.wq_tensors(lq.lq_pack_weights(dev(w)))
+        torch.cuda.synchronize()
+        assert host(sc)[0, 0] == np.float32(case["scale"])
+        codes = O.unpack_int4(host(c4))[0]
+        assert list(codes[:len(case["codes"])]) == case["codes"]
+        assert not codes[len(case["codes"]):].any()
+    for case in gold["packing_cases"]:
+        # weights equal to the codes themselves: step 1 when the absmax is 7
+        w = np.zeros((1, 32), np.float32)
+        w[0, :len(case["codes"])] = case["codes"]
+        c4, _ = lq.wq_tensors(lq.lq_pack_weights(dev(w)))
+        torch.cuda.synchronize()
+        assert list(host(c4)[0, :len(case["bytes"])]) == case["bytes"]

@@ -185,6 +185,19 @@ def pin_kron(o):
             want[m, col] = tot
     got = o.kron_rotate(xs, A, B)
     assert np.max(np.abs(got - want)) <= 1e-5
+    # rounded once: each element is the float32 nearest to the exact rational
+    # sum (float64 arithmetic is 2^-29 closer than float32's half-ulp, so a
+    # double rounding could only differ within 2^-29 ulp of a tie; none is)
+    for m in range(2):
+        for col in range(12):
+            i, j = divmod(col, 4)
+            exact = sum(Fraction(float(xs[m, row])) * Fraction(float(A[row // 4, i]))
+                        * Fraction(float(B[row % 4, j])) for row in range(12))
+            below = np.float32(float(exact))
+            cands = [below, np.nextafter(below, np.float32(np.inf)),
+                     np.nextafter(below, np.float32(-np.inf))]
+            nearest = min(cands, key=lambda c: abs(Fraction(float(c)) - exact))
+            assert got[m, col] == nearest, (m, col)
     # P1 = swap, P2 = I maps [x0,x1,x2,x3] -> [x2,x3,x0,x1]
     v = np.array([[1.0, 2.0, 3.0, 4.0]], np.float32)
     swap = np.array([[0, 1], [1, 0]], np.float32)
@@ -444,6 +457,18 @@ def _runs_all(o):
         pin(o)
 
 
+def _gemm_fold_f32(qa, sa, qw, sw, group=32):
+    """The group fold y += (s_a s_w) acc carried in float32 instead of float64."""
+    qa = np.asarray(qa).astype(np.float32)
+    qw = np.asarray(qw).astype(np.float32)
+    G = qa.shape[1] // group
+    y = np.zeros((qa.shape[0], qw.shape[0]), np.float32)
+    for g in range(G):
+        acc = qa[:, g * group:(g + 1) * group] @ qw[:, g * group:(g + 1) * group].T
+        y += (np.asarray(sa, np.float32)[:, g][:, None] * np.asarray(sw, np.float32)[:, g][None, :]) * acc
+    return y.astype(np.float64)
+
+
 MUTANTS = {
     "ties_away_from_zero": dict(quantize_groups=_q_variant(
         rounding=lambda r: np.sign(r) * np.floor(np.abs(r) + 0.5))),
@@ -463,6 +488,12 @@ MUTANTS = {
                                     O.group_gemm(qa, sa, qw, np.ones_like(sw), group)),
     "gemm_groups_misaligned": dict(group_gemm=lambda qa, sa, qw, sw, group=32:
                                    O.group_gemm(qa, sa[:, ::-1], qw, sw, group)),
+    "quotient_by_reciprocal_multiply": dict(quantize_groups=_q_variant(divide=False)),
+    "rotation_accumulated_in_float32": dict(kron_rotate=lambda x, P1, P2: np.einsum(
+        "pi,mpq,qj->mij", np.asarray(P1, np.float32),
+        np.asarray(x, np.float32).reshape(len(x), P1.shape[0], P2.shape[0]),
+        np.asarray(P2, np.float32)).reshape(len(x), -1).astype(np.float32)),
+    "gemm_fold_in_float32": dict(group_gemm=_gemm_fold_f32),
 }
 
 
