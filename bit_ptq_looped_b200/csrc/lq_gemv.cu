@@ -565,7 +565,7 @@ cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa
   // 2 to 4 tokens: dp4a while the rows fit in about one resident wave of
   // warps (one memory latency per warp, the decode-sized launches); once the
   // launch streams at least a wave of 16-row blocks, the tensor-core path
-  // with its deeper weight pipeline (a 263 MB launch at M = 4: 5.3 TB/s
+  // with its deeper weight pipeline (a 263 MB launch at M = 4: 5.5 TB/s
   // against 2.9 with dp4a)
   if (M <= 4 && N < (int64_t)num_sms() * 2 * kMmaWarps * 16)
     return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
