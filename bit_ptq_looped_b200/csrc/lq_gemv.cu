@@ -24,9 +24,11 @@
 // under programmatic dependent launch the weight stream of this launch
 // overlaps the quantizer that produces its activation.
 #include <algorithm>
+#include <map>
 #include <mutex>
+#include <set>
+#include <tuple>
 #include <type_traits>
-#include <unordered_map>
 
 #include "lq_common.cuh"
 
@@ -431,35 +433,48 @@ size_t gemv_smem_bytes(int64_t M, int64_t G) { return (size_t)M * G * (32 + 8); 
 constexpr size_t kGemvMaxSmem = 200u * 1024u;  // the activation bound of the GEMV path
 constexpr size_t kMmaMaxSmem = 227u * 1024u;   // opt-in shared memory of one block
 
+// Resident blocks per SM of kernel k with `smem` bytes of dynamic shared memory
+// on the current device.  The first query for a (device, kernel) raises the
+// kernel's limit there to max_smem, the largest size any call uses, so that it
+// is never lowered under a launch recorded earlier; results are cached.
+template <typename F>
+cudaError_t blocks_per_sm(F* k, int threads, size_t smem, size_t max_smem, int* per_sm) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, size_t>, int> cache;
+  static std::set<std::pair<int, const void*>> raised;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_tuple(dev, (const void*)k, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *per_sm = it->second;
+    return cudaSuccess;
+  }
+  if (!raised.count({dev, (const void*)k})) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+    if (e != cudaSuccess) return e;
+    raised.insert({dev, (const void*)k});
+  }
+  int n = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem);
+  if (e != cudaSuccess) return e;
+  if (n < 1) return cudaErrorInvalidConfiguration;
+  cache.emplace(key, n);
+  *per_sm = n;
+  return cudaSuccess;
+}
+
 template <int MB, int GPL, int RPW, bool kDB>
 cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                        const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
                        bool pdl) {
   const size_t smem = gemv_smem_bytes(M, K / kGroup);
   auto* k = k_group_gemv<MB, GPL, RPW, kDB>;
-  // resident blocks per SM for this instantiation and shared-memory size
-  static std::mutex mu;
-  static std::unordered_map<size_t, int> per_sm_cache;
   int per_sm = 0;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = per_sm_cache.find(smem);
-    if (it == per_sm_cache.end()) {
-      // the attribute is one per function: raise it once to the largest activation
-      // any call can stage, never lower it under an earlier call's size
-      if (per_sm_cache.empty()) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kGemvMaxSmem);
-        if (e != cudaSuccess) return e;
-      }
-      cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemvThreads, smem);
-      if (e != cudaSuccess) return e;
-      if (per_sm < 1) return cudaErrorInvalidConfiguration;
-      per_sm_cache.emplace(smem, per_sm);
-    } else {
-      per_sm = it->second;
-    }
-  }
+  cudaError_t e = blocks_per_sm(k, kGemvThreads, smem, kGemvMaxSmem, &per_sm);
+  if (e != cudaSuccess) return e;
   // enough warps for one batch of RPW rows each, capped at one resident wave
   const int64_t warps_needed = (N + RPW - 1) / RPW;
   const int64_t want = (warps_needed + kGemvWarps - 1) / kGemvWarps;
@@ -487,28 +502,9 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
   const size_t smem = mma_act_bytes(NB, G) + (size_t)kMmaWarps * kS * mma_stage_bytes(kU);
   if (smem > kMmaMaxSmem) return cudaErrorInvalidValue;
   auto* k = k_group_gemv_mma<NB, kS, kU, 2>;
-  static std::mutex mu;
-  static std::unordered_map<size_t, int> per_sm_cache;
   int per_sm = 0;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = per_sm_cache.find(smem);
-    if (it == per_sm_cache.end()) {
-      // one attribute per function: raised once to the largest size any call uses
-      if (per_sm_cache.empty()) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kMmaMaxSmem);
-        if (e != cudaSuccess) return e;
-      }
-      cudaError_t e =
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kMmaWarps * 32, smem);
-      if (e != cudaSuccess) return e;
-      if (per_sm < 1) return cudaErrorInvalidConfiguration;
-      per_sm_cache.emplace(smem, per_sm);
-    } else {
-      per_sm = it->second;
-    }
-  }
+  cudaError_t e = blocks_per_sm(k, kMmaWarps * 32, smem, kMmaMaxSmem, &per_sm);
+  if (e != cudaSuccess) return e;
   const int64_t row_blocks = (N + 15) / 16;
   const int64_t want = (row_blocks + kMmaWarps - 1) / kMmaWarps;
   const int64_t blocks = std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
