@@ -18,6 +18,7 @@
 // turn, and writes a*h + b + eta * (p U^T) from the accumulator fragments.  U
 // and V are held as float64 d x 8 (rank padded with zero columns).
 #include <algorithm>
+#include <atomic>
 
 #include "lq_common.cuh"
 
@@ -122,14 +123,14 @@ cudaError_t launch_cta_apply(const float* h, int64_t M, int d, const double* U8,
   if (M == 0) return cudaSuccess;
   const size_t smem = cta_smem_bytes(d);
   if (d % 32 || smem > 200u * 1024u) return cudaErrorInvalidValue;
-  static int attr_dev_mask = 0;
+  static std::atomic<uint64_t> attr_dev_mask{0};  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!((attr_dev_mask >> (dev & 31)) & 1)) {
+  if (!((attr_dev_mask.load() >> (dev & 63)) & 1u)) {
     cudaError_t e = cudaFuncSetAttribute(k_cta_apply, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          200 * 1024);
     if (e != cudaSuccess) return e;
-    attr_dev_mask |= 1 << (dev & 31);
+    attr_dev_mask.fetch_or(1ull << (dev & 63));
   }
   const int64_t want = (M + 7) / 8;
   const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * 8);

@@ -513,16 +513,14 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
 }
 
 // the tensor-core GEMV for M tokens: one block of 8 tokens with 16-group
-// stages (2 in flight per warp), or two blocks with 8-group stages (3, or 2
-// when the activation leaves too little shared memory for 3)
+// stages (2 in flight per warp), or two blocks with 8-group stages (3 in
+// flight); the activation and the rings fit a block's shared memory up to
+// K = 8544 at 16 tokens, above every Kronecker shape the rotation stages
 cudaError_t launch_tc(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                       const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
                       bool pdl) {
-  const int64_t G = K / kGroup;
   if (M <= 8) return launch_mma<1, 2, 16>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  if (mma_act_bytes(2, G) + (size_t)kMmaWarps * 3 * mma_stage_bytes(8) <= kMmaMaxSmem)
-    return launch_mma<2, 3, 8>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  return launch_mma<2, 2, 8>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_mma<2, 3, 8>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
 
 template <int MB>
