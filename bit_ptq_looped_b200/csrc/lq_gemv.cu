@@ -515,7 +515,7 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
 // the tensor-core GEMV for M tokens: one block of 8 tokens with 16-group
 // stages (2 in flight per warp), or two blocks with 8-group stages (3 in
 // flight); the activation and the rings fit a block's shared memory up to
-// K = 8544 at 16 tokens, above every Kronecker shape the rotation stages
+// K = 8544 at 16 tokens, above the K <= 8192 of the GEMV path
 cudaError_t launch_tc(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                       const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
                       bool pdl) {
