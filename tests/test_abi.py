@@ -129,3 +129,49 @@ def test_inverse_transpose_host_helper():
         assert np.max(np.abs(got - want)) <= 1e-6 * max(1.0, np.max(np.abs(want)))
     with pytest.raises(lq.LQError):
         lq.lq_inverse_transpose(np.zeros((3, 3), np.float32))
+
+
+def test_size_functions(L):
+    # lq_act_scale_bytes: one float32 step per row and group of 32
+    for M, K in ((1, 32), (7, 2048), (2048, 5632)):
+        assert L.lq_act_scale_bytes(M, K) == M * (K // 32) * 4
+    # lq_hessian_workspace_bytes: the transposed bf16 inputs, K x (M*T rows, padded), 256-aligned
+    assert L.lq_hessian_workspace_bytes(-1, 128, 1) == -1
+    assert L.lq_hessian_workspace_bytes(4, 0, 1) == -1
+    assert L.lq_hessian_workspace_bytes(4, 128, 0) == -1
+    prev = 0
+    for M, K, T in ((1, 128, 1), (5, 256, 4), (2048, 2048, 4), (2049, 2048, 4)):
+        n = L.lq_hessian_workspace_bytes(M, K, T)
+        assert n >= K * M * T * 2 and n % 256 == 0
+        assert n < K * (M * T + 64) * 2 + 256  # padding below one 64-row block
+        assert n >= prev
+        prev = n
+
+
+def test_hessian_entry_rejects_bad_arguments(L):
+    fake = 1 << 20  # never dereferenced: every call below fails its checks first
+    big = 1 << 40
+    # inputs must be bf16
+    assert L.lq_trajectory_hessian(fake, lq.LQ_F32, 4, 128, 2, fake, 0, fake, big, None) == \
+        lq.LQ_ERR_UNSUPPORTED
+    # shapes
+    assert L.lq_trajectory_hessian(fake, lq.LQ_BF16, -1, 128, 2, fake, 0, fake, big, None) == \
+        lq.LQ_ERR_ARG
+    assert L.lq_trajectory_hessian(fake, lq.LQ_BF16, 4, 128, 0, fake, 0, fake, big, None) == \
+        lq.LQ_ERR_ARG
+    assert L.lq_trajectory_hessian(fake, lq.LQ_BF16, 4, 100, 2, fake, 0, fake, big, None) == \
+        lq.LQ_ERR_SHAPE
+    # H: null, misaligned
+    assert L.lq_trajectory_hessian(fake, lq.LQ_BF16, 4, 128, 2, None, 0, fake, big, None) == \
+        lq.LQ_ERR_ARG
+    assert L.lq_trajectory_hessian(fake, lq.LQ_BF16, 4, 128, 2, fake + 4, 0, fake, big, None) == \
+        lq.LQ_ERR_ALIGN
+    # no rows while accumulating: H stays as it is, nothing is enqueued
+    assert L.lq_trajectory_hessian(None, lq.LQ_BF16, 0, 128, 2, fake, 1, None, 0, None) == lq.LQ_OK
+    # X and workspace: null, misaligned, too small
+    assert L.lq_trajectory_hessian(None, lq.LQ_BF16, 4, 128, 2, fake, 0, fake, big, None) == \
+        lq.LQ_ERR_ARG
+    assert L.lq_trajectory_hessian(fake, lq.LQ_BF16, 4, 128, 2, fake, 0, fake + 16, big, None) == \
+        lq.LQ_ERR_ALIGN
+    assert L.lq_trajectory_hessian(fake, lq.LQ_BF16, 4, 128, 2, fake, 0, fake, 256, None) == \
+        lq.LQ_ERR_WORKSPACE
