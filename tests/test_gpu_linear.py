@@ -186,6 +186,11 @@ def _stack_inputs(wl, M):
 @pytest.mark.parametrize("wl,M", [(synth.TINY, 64), (synth.MLP, 384), (synth.ATTN_PROJ, 2048)],
                          ids=["tiny", "mlp", "attn"])
 def test_loop_stack_open(wl, M):
+    """Open-mode stack with the default workspace, sized for all T loops: at
+    attn (M = K = N = 2048, T = 4, W4A4) this is the benchmark's timed
+    configuration, one rotate+quantize launch and one GEMM launch for the 4
+    loops; every output of every loop against the oracle, and graph replays
+    bit-identical."""
     params = synth.module_params(wl)
     built = [make_layer(mp, wl.a_bits) for mp in params]
     layers = [b[0] for b in built]
