@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kGemvThreads, kDB ? 1 : 3) k_group_gemv(
 //
 // Weight stream.  Each warp owns a ring of kS shared-memory stages; a stage is
 // 16 rows x kU groups of packed codes (16 bytes per row and group) plus their
-// steps, brought in by cp.async (the 8 lanes of a row copy 128 contiguous
+// steps, brought in by cp.async (kU lanes copy a row's kU * 16 contiguous
 // bytes) and read back with ldmatrix, which hands thread (g, t) word t of row
 // g: the A fragment, transposed in the load.  Chunks are stored XOR-swizzled
 // by row so that the 8 row addresses of an ldmatrix hit distinct banks.  The
