@@ -277,9 +277,38 @@ def pin_special_cases(o):
                           (qa.astype(np.int64) @ qw.astype(np.int64).T).astype(np.float64))
 
 
+def pin_loop_clip_index(o):
+    """Loop t quantizes with its own clip c_t = las[t] (paper_specification.yaml:
+    las, c_{t,l} per module and loop): a hand-worked case with four distinct
+    clips, identity transforms and an exactly quantizable weight, through both
+    the single-step call and the open- and chain-mode drivers."""
+    (case,) = _golden()["loop_cases"]
+    K, n = case["K"], len(case["x"])
+    T = len(case["las"])
+    W = np.float32(0.875) * np.eye(K, dtype=np.float32)
+    layer = o.OracleLayer(W, np.eye(case["a"], dtype=np.float32),
+                          np.eye(case["b"], dtype=np.float32),
+                          np.asarray(case["las"], np.float32), 4)
+    x = _pad32(case["x"])
+    ys = o.loop_stack_open([[x] for _ in range(T)], [layer], T)
+    for t in range(T):
+        want = np.zeros((1, K))
+        want[0, :n] = case["y"][t]
+        assert np.array_equal(ys[t][0], want), f"loop {t}"
+        assert np.array_equal(o.loop_linear(x, layer, t), want), f"loop {t}"
+    # chain mode feeds y back; loop 1 must still clip with c_1 (its input is
+    # loop 0's output, 0.875 * the codes of case w4a4_c1: absmax 6.125)
+    ch = o.loop_stack_chain(x, [layer], 2)
+    y0 = ch[0][0].astype(np.float32)
+    s1 = np.float32(np.float32(case["las"][1]) * np.float32(6.125)) / np.float32(7)
+    assert s1 == np.float32(0.4375)
+    q1 = np.clip(np.rint(y0 / s1), -7, 7)  # y0 / s1 = 2 * the t = 0 codes, no ties
+    assert np.array_equal(ch[1][0], 0.875 * np.float64(s1) * q1.astype(np.float64))
+
+
 ALL_PINS = [pin_hand_activation, pin_hand_weight, pin_hand_packing, pin_hand_gemm,
             pin_rtn_bruteforce, pin_invariants, pin_kron, pin_fold_invariance,
-            pin_gemm_bruteforce, pin_special_cases]
+            pin_gemm_bruteforce, pin_special_cases, pin_loop_clip_index]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
@@ -469,6 +498,23 @@ def _gemm_fold_f32(qa, sa, qw, sw, group=32):
     return y.astype(np.float64)
 
 
+class _LayerFirstClip(O.OracleLayer):
+    """Planted mistake: every loop quantizes with the clip of loop 0."""
+
+    def forward(self, x, t):
+        qa, sa = O.quantize_activation(x, self.P1, self.P2, float(self.las[0]), self.a_bits)
+        return O.group_gemm(qa, sa, self.qw, self.sw)
+
+
+class _LayerNextClip(O.OracleLayer):
+    """Planted mistake: loop t quantizes with the clip of loop t + 1 (wrapping)."""
+
+    def forward(self, x, t):
+        c = float(self.las[(t + 1) % self.las.size])
+        qa, sa = O.quantize_activation(x, self.P1, self.P2, c, self.a_bits)
+        return O.group_gemm(qa, sa, self.qw, self.sw)
+
+
 MUTANTS = {
     "ties_away_from_zero": dict(quantize_groups=_q_variant(
         rounding=lambda r: np.sign(r) * np.floor(np.abs(r) + 0.5))),
@@ -494,6 +540,8 @@ MUTANTS = {
         np.asarray(x, np.float32).reshape(len(x), P1.shape[0], P2.shape[0]),
         np.asarray(P2, np.float32)).reshape(len(x), -1).astype(np.float32)),
     "gemm_fold_in_float32": dict(group_gemm=_gemm_fold_f32),
+    "loop_uses_first_clip": dict(OracleLayer=_LayerFirstClip),
+    "loop_uses_next_loop_clip": dict(OracleLayer=_LayerNextClip),
 }
 
 
