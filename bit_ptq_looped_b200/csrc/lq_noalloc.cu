@@ -22,10 +22,31 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LQ_NOALLOC_SCRA
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchEntry {
+  void* ctx;  // the context the address belongs to
+  void* ptr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
+using CtxGetCurrentFn = int (*)(void**);  // cuCtxGetCurrent(CUcontext*)
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch on the current device, looked up with that
+// device current and cached per device together with the context it belongs
+// to: after a device reset (a new primary context, the module loaded again,
+// possibly elsewhere) the address is looked up again.
 lq_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -34,14 +55,24 @@ lq_status scratch_address(void** out) {
     set_error("device index %d out of range", dev);
     return LQ_ERR_ARG;
   }
+  e = cudaSetDevice(dev);  // the same device: makes its primary context current
+  if (e != cudaSuccess) return cuda_error(e, "cudaSetDevice");
+  CtxGetCurrentFn get = ctx_get_current();
+  void* ctx = nullptr;
+  if (get == nullptr || get(&ctx) != 0 || ctx == nullptr) {
+    set_error("cannot query the current CUDA context");
+    return LQ_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchEntry& ent = g_scratch[dev];
+  if (ent.ptr == nullptr || ent.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress of the static scratch");
-    g_scratch_ptr[dev] = p;
+    ent.ctx = ctx;
+    ent.ptr = p;
   }
-  *out = g_scratch_ptr[dev];
+  *out = ent.ptr;
   return LQ_OK;
 }
 

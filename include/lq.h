@@ -326,8 +326,9 @@ lq_status lq_trajectory_hessian(const void* d_X, int32_t x_dtype, int64_t M, int
  *     (for instance on two streams without ordering between them) race on the
  *     array and give wrong results.
  *   - The first call on a device looks the array's device address up (once
- *     per device, with that device current); make that first call before any
- *     stream capture.
+ *     per device and context, with that device current); make that first
+ *     call before any stream capture.  After a device reset the next call
+ *     looks the address up again, so make it outside a capture too.
  */
 #define LQ_NOALLOC_SCRATCH_BYTES (16ll << 20)
 lq_status lq_loop_linear_noalloc(const void* d_x, int32_t x_dtype, int64_t M,

@@ -183,13 +183,14 @@ def _stack_inputs(wl, M):
     return xs, flat
 
 
-@pytest.mark.parametrize("wl,M", [(synth.TINY, 64), (synth.MLP, 384), (synth.ATTN_PROJ, 2048)],
+@pytest.mark.parametrize("wl,M", [(synth.TINY, 64), (synth.MLP, 2048), (synth.ATTN_PROJ, 2048)],
                          ids=["tiny", "mlp", "attn"])
 def test_loop_stack_open(wl, M):
-    """Open-mode stack with the default workspace, sized for all T loops: at
-    attn (M = K = N = 2048, T = 4, W4A4) this is the benchmark's timed
-    configuration, one rotate+quantize launch and one GEMM launch for the 4
-    loops; every output of every loop against the oracle, and graph replays
+    """Open-mode stack with the default workspace, sized for all T loops: one
+    rotate+quantize launch and one GEMM launch per linear for the 4 loops (the
+    launch configuration the benchmark times for these workloads, at their full
+    sizes: M = 2048; the MLP's down projection runs 8192 rows of K = 5632 per
+    launch); every output of every loop against the oracle, and graph replays
     bit-identical."""
     params = synth.module_params(wl)
     built = [make_layer(mp, wl.a_bits) for mp in params]
@@ -400,3 +401,52 @@ def test_calib_block_full_size_sampled_rows():
             linear_parity(ys, xs, ol, t, host(q8), host(s), layer.w_flips)
             del x
         lq.lq_check_device()
+
+
+def test_calib_block_stack_full_size_sampled_rows():
+    """The benchmark's headline step at full size: lq_loop_stack in open mode
+    over the 7 shared linears x T = 4 loops on M = 262144 tokens, with the
+    workspace that batches the 4 loops of a linear into one quantize and one
+    GEMM launch (1048576 rows per launch).  Every (module, loop) output is
+    checked against the oracle on sampled rows (rows are independent): the
+    first and last rows, rows at 128-row tile and 256-row block edges, and
+    random rows."""
+    wl = synth.CALIB_BLOCK
+    params = synth.module_params(wl)
+    M, T = wl.M, wl.T
+    built = [make_layer(mp, wl.a_bits) for mp in params]
+    layers = [b[0] for b in built]
+    rng = np.random.default_rng(17)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, 255, 256, M // 2 - 1, M // 2, M - 129,
+                                      M - 128, M - 1], rng.choice(M, 53, replace=False)]))
+    rows_d = torch.from_numpy(rows).cuda()
+    sum_k = sum(lin.K for lin in wl.linears)
+    sum_n = sum(lin.N for lin in wl.linears)
+    x = torch.empty(T * M * sum_k, dtype=torch.bfloat16, device="cuda")
+    off = 0
+    for t in range(T):
+        for lin in wl.linears:
+            x[off:off + M * lin.K] = synth.device_loop_input(wl, lin, t).reshape(-1)
+            off += M * lin.K
+    y = torch.empty(T * M * sum_n, dtype=torch.float32, device="cuda")
+    ws = lq.workspace(layers, M, T=T)
+    lq.lq_loop_stack(x, layers, T, lq.LQ_OPEN, M=M, y=y, ws=ws)
+    torch.cuda.synchronize()
+    lq.lq_check_device()
+    del ws
+    xo = yo = 0
+    for t in range(T):
+        for l, (lin, mp) in enumerate(zip(wl.linears, params)):
+            xs = x[xo:xo + M * lin.K].view(M, lin.K)[rows_d].contiguous()
+            ys = host(y[yo:yo + M * lin.N].view(M, lin.N)[rows_d])
+            xo += M * lin.K
+            yo += M * lin.N
+            q8, _, s = lq.lq_quantize_act(xs, dev(mp.P1), dev(mp.P2), float(mp.las[t]),
+                                          wl.a_bits)
+            torch.cuda.synchronize()
+            linear_parity(ys, xs.float().cpu().numpy(), built[l][1], t, host(q8), host(s),
+                          built[l][0].w_flips)
+    del x, y
+    for layer, _ in built:
+        layer.free()
+    torch.cuda.empty_cache()
