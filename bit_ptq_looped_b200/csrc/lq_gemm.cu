@@ -440,17 +440,26 @@ __global__ void k_wait_selftest(uint64_t limit_ns) {
 // index is contiguous.  Then H = Xt Xt^T on the tensor cores: one CTA per
 // 128 x 128 tile of the upper triangle (the lower one is its mirror), a TMA
 // warp streaming 128 x 64 bf16 tiles of both row blocks through a 6-stage
-// ring, an MMA warp issuing four kind::f16 MMAs (K = 16 each) per stage into
-// one float32 TMEM accumulator that runs over the whole reduction, and four
-// epilogue warps writing the tile and, off the diagonal, its transpose.
-// bf16 products are exact in float32; the sums are the tensor core's float32
-// accumulation.
+// ring, an MMA warp issuing four kind::f16 MMAs (K = 16 each) per stage, and
+// four epilogue warps.  bf16 products are exact in float32; what rounds is
+// the summation.  The tensor core's float32 accumulation loses up to about
+// one unit in the last place per MMA (it does not round to nearest), which
+// over a reduction of thousands of rows grows into a relative error of some
+// 1e-5.  So the reduction is cut into slices of 256 rows (16 MMAs): each slice
+// is summed by the tensor core into its own TMEM accumulator (four rotate
+// through the 512 columns, so the tensor core runs up to three slices ahead),
+// and the epilogue adds the finished slices, in order, into float32 registers
+// (round to nearest), then writes the tile and, off the diagonal, its
+// transpose.
 // ---------------------------------------------------------------------------
 namespace {
 
 constexpr int HT = 128;               // tile rows / columns of H
 constexpr int HK = 64;                // reduction elements per stage (128-byte bf16 rows)
 constexpr int H_STAGES = 6;
+constexpr int H_SLICE_STAGES = 4;     // stages per accumulator slice: 256 rows, 16 MMAs
+constexpr int H_ACC_BUFS = 4;         // 4 x 128 TMEM columns
+constexpr int H_TMEM_COLS = HT * H_ACC_BUFS;
 constexpr uint32_t H_TILE_BYTES = HT * HK * 2;  // 16 KB
 constexpr uint32_t H_STAGE_TX = 2 * H_TILE_BYTES;
 constexpr int H_EPI_WARPS = 4;
@@ -459,7 +468,8 @@ constexpr int H_THREADS = 32 * (H_EPI_WARPS + 2);
 constexpr uint32_t H_OFF_A = 0;
 constexpr uint32_t H_OFF_B = H_OFF_A + H_STAGES * H_TILE_BYTES;
 constexpr uint32_t H_OFF_BAR = H_OFF_B + H_STAGES * H_TILE_BYTES;
-constexpr uint32_t H_N_BARS = 2 * H_STAGES + 2;  // full, empty, accumulator full, drain
+// full, empty per stage; accumulator full, empty per slice buffer; drain
+constexpr uint32_t H_N_BARS = 2 * H_STAGES + 2 * H_ACC_BUFS + 1;
 constexpr uint32_t H_OFF_MISC = H_OFF_BAR + H_N_BARS * 8;
 constexpr uint32_t H_SMEM_BYTES = H_OFF_MISC + 16 + 1024;
 
@@ -500,10 +510,12 @@ __global__ void __launch_bounds__(H_THREADS, 1)
   const uint32_t bar_full = base + H_OFF_BAR;
   const uint32_t bar_empty = bar_full + H_STAGES * 8;
   const uint32_t bar_accf = bar_empty + H_STAGES * 8;
-  const uint32_t bar_drain = bar_accf + 8;
+  const uint32_t bar_acce = bar_accf + H_ACC_BUFS * 8;
+  const uint32_t bar_drain = bar_acce + H_ACC_BUFS * 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + H_OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + H_OFF_MISC + 4);
   const int nt = K / HT;
+  const int n_slices = (n_kb + H_SLICE_STAGES - 1) / H_SLICE_STAGES;
   int mb, nb;
   upper_tile(blockIdx.x, nt, mb, nb);
   const int m0 = mb * HT, n0 = nb * HT;
@@ -514,14 +526,17 @@ __global__ void __launch_bounds__(H_THREADS, 1)
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_accf, 1);
+    for (int b = 0; b < H_ACC_BUFS; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, H_EPI_WARPS);
+    }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == H_WARP_TMA && lane == 0) prefetch_tmap(&tmX);
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), HT);
+    tmem_alloc(smem_u32(tmem_slot), H_TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -552,23 +567,35 @@ __global__ void __launch_bounds__(H_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc_bf16();
       bool ok = true;
-      for (int kb = 0; kb < n_kb; ++kb) {
-        const int st = kb % H_STAGES;
-        if (!mbar_wait_bounded(bar_full + 8 * st, (uint32_t)(kb / H_STAGES) & 1u, abort_flag,
-                               &g_gemm_status, kWaitLimitNs)) {
+      for (int j = 0; j < n_slices && ok; ++j) {
+        const int buf = j % H_ACC_BUFS;
+        // the epilogue has read this buffer's previous slice
+        if (!mbar_wait_bounded(bar_acce + 8 * buf, ((uint32_t)(j / H_ACC_BUFS) & 1u) ^ 1u,
+                               abort_flag, &g_gemm_status, kWaitLimitNs)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_st = base + H_OFF_A + st * H_TILE_BYTES;
-        const uint32_t b_st = base + H_OFF_B + st * H_TILE_BYTES;
+        const uint32_t d = tmem_base + (uint32_t)(buf * HT);
+        const int kb_end = min(n_kb, (j + 1) * H_SLICE_STAGES);
+        for (int kb = j * H_SLICE_STAGES; kb < kb_end; ++kb) {
+          const int st = kb % H_STAGES;
+          if (!mbar_wait_bounded(bar_full + 8 * st, (uint32_t)(kb / H_STAGES) & 1u, abort_flag,
+                                 &g_gemm_status, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_st = base + H_OFF_A + st * H_TILE_BYTES;
+          const uint32_t b_st = base + H_OFF_B + st * H_TILE_BYTES;
 #pragma unroll
-        for (int j = 0; j < HK / 16; ++j)  // K = 16 bf16 = 32 bytes per MMA
-          umma_bf16(tmem_base, sw128_kmajor_desc(a_st + 32u * j),
-                    sw128_kmajor_desc(b_st + 32u * j), idesc, (kb | j) != 0 ? 1u : 0u);
-        umma_commit(bar_empty + 8 * st);
+          for (int i = 0; i < HK / 16; ++i)  // K = 16 bf16 = 32 bytes per MMA
+            umma_bf16(d, sw128_kmajor_desc(a_st + 32u * i), sw128_kmajor_desc(b_st + 32u * i),
+                      idesc, (kb > j * H_SLICE_STAGES || i != 0) ? 1u : 0u);
+          umma_commit(bar_empty + 8 * st);
+        }
+        if (ok) umma_commit(bar_accf + 8 * buf);
       }
-      if (ok) umma_commit(bar_accf);
       umma_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0u);
     }
@@ -576,37 +603,51 @@ __global__ void __launch_bounds__(H_THREADS, 1)
     // ---- epilogue: warp q reads TMEM lanes 32q..32q+31 = rows m0 + 32q + lane
     const int q = warp;
     const int row = q * 32 + lane;
-    pdl_wait();  // H may be read by an earlier kernel of the stream
-    if (mbar_wait_bounded(bar_accf, 0u, abort_flag, &g_gemm_status, kWaitLimitNs)) {
+    const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
+    float h[HT];
+#pragma unroll
+    for (int i = 0; i < HT; ++i) h[i] = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_slices && ok; ++j) {
+      const int buf = j % H_ACC_BUFS;
+      ok = mbar_wait_bounded(bar_accf + 8 * buf, (uint32_t)(j / H_ACC_BUFS) & 1u, abort_flag,
+                             &g_gemm_status, kWaitLimitNs);
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < HT / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(lane_base + (uint32_t)(32 * c), r);
+        tmem_ld_32x32b_x32(lane_base + (uint32_t)(buf * HT + 32 * c), r);
         tmem_wait_ld();
-        // tile (m0 + row, n0 + 32c + i): each thread writes 32 consecutive floats of its row
-        float* dst = H + (size_t)(m0 + row) * K + n0 + 32 * c;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float4 v = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                 __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-          if (accumulate) {
-            const float4 o = *reinterpret_cast<const float4*>(dst + i);
-            v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
-          }
-          *reinterpret_cast<float4*>(dst + i) = v;
+        for (int i = 0; i < 32; ++i) h[32 * c + i] += __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acce + 8 * buf);
+    }
+    pdl_wait();  // H may be read by an earlier kernel of the stream
+    if (ok) {
+      // tile (m0 + row, n0 + i): each thread writes the 128 consecutive floats of its row
+      float* dst = H + (size_t)(m0 + row) * K + n0;
+#pragma unroll
+      for (int i = 0; i < HT; i += 4) {
+        float4 v = make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]);
+        if (accumulate) {
+          const float4 o = *reinterpret_cast<const float4*>(dst + i);
+          v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
         }
-        if (nb != mb) {
-          // mirrored tile (n0 + 32c + i, m0 + row): for each i the 32 lanes write 32
-          // consecutive floats
+        *reinterpret_cast<float4*>(dst + i) = v;
+      }
+      if (nb != mb) {
+        // mirrored tile (n0 + i, m0 + row): for each i the 32 lanes write 32
+        // consecutive floats
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float* md = H + (size_t)(n0 + 32 * c + i) * K + m0 + row;
-            float v = __uint_as_float(r[i]);
-            if (accumulate) v += *md;
-            *md = v;
-          }
+        for (int i = 0; i < HT; ++i) {
+          float* md = H + (size_t)(n0 + i) * K + m0 + row;
+          float v = h[i];
+          if (accumulate) v += *md;
+          *md = v;
         }
       }
     }
@@ -615,7 +656,7 @@ __global__ void __launch_bounds__(H_THREADS, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, HT);
+    tmem_dealloc(tmem_base, H_TMEM_COLS);
   }
 }
 

@@ -7,7 +7,10 @@ Tolerances (stated for the quantized looped linear):
     divided by the step lies within 1e-6 (relative) of a rounding tie k + 1/2;
   * GEMM: max|dy| <= 1e-3 max|y| and relative L2 <= 1e-5 against the float64
     oracle, on rows whose codes agree; rows holding an allowed near-tie code
-    difference are checked against the bound that difference implies.
+    difference are checked against the bound that difference implies;
+  * trajectory Hessian (bf16 inputs, products exact in float32): relative
+    Frobenius error <= 1e-5 of ||H||, and every element within the bound of
+    the kernel's summation (see check_hessian).
 """
 import numpy as np
 import torch
@@ -115,3 +118,31 @@ def linear_parity(y_gpu, x, ol, t, q_gpu, s_gpu, w_flips=None):
     tol = 1e-3 * np.abs(y_or).max()
     assert np.all(np.abs(y_gpu - y_or) <= bound + tol)
     return y_or, len(flips)
+
+
+# rows per accumulator slice of the Hessian kernel and MMAs (K = 16) per slice
+HESSIAN_SLICE_ROWS = 256
+HESSIAN_MMAS_PER_SLICE = HESSIAN_SLICE_ROWS // 16
+
+
+def hessian_bound(A, n_rows):
+    """Element bound of the kernel's float32 summation of n_rows exact
+    products: each slice of 256 rows is summed by the tensor core (16 MMAs;
+    allowed 2^-21 of the running sum of magnitudes per MMA, four units in the
+    last place, since the tensor core's accumulation does not round to
+    nearest), then the n_slices partial sums (and H0 when accumulating) are
+    added in float32 with round to nearest (2^-24 per addition).  A is the sum
+    of |x_i x_j| (plus |H0|)."""
+    n_slices = -(-n_rows // HESSIAN_SLICE_ROWS)
+    return (HESSIAN_MMAS_PER_SLICE * 2.0 ** -21 + (n_slices + 2) * 2.0 ** -24) * A
+
+
+def check_hessian(Hg, Hor, A, n_rows):
+    """Hg (the library's H or rows of it) against the float64 oracle Hor."""
+    Hg = np.asarray(Hg, np.float64)
+    err = np.abs(Hg - Hor)
+    bound = hessian_bound(A, n_rows)
+    assert np.all(err <= bound + 1e-30), f"max err/bound {(err / (bound + 1e-300)).max()}"
+    rel = np.linalg.norm(err) / max(np.linalg.norm(Hor), 1e-300)
+    assert rel <= 1e-5, f"relative Frobenius error {rel}"
+    return rel
