@@ -531,6 +531,263 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
 }
 
 // ---------------------------------------------------------------------------
+// Warp-specialised fused rotation + quantization for many token rows.
+//
+// The same arithmetic as k_rotate_quant (X -> X P2 -> P1^T (X P2) on the
+// FP64 tensor-core MMA, float64 sums rounded once to float32, then the
+// group-32 quantizer), but the FP64 MMA never waits for the quantizer: one
+// persistent block per SM runs
+//   8 MMA warps   stage 1 into YT, stage 2 into Z (written over the tile's X),
+//   4 quant warps staging the next tiles' inputs into shared memory and
+//                 quantizing the finished Z tiles,
+// over two X/Z tile buffers.  Per tile i (buffer s = i % 2) the quant warps
+// load X(i) into buffer s and arrive on barrier XFULL[s]; the MMA warps wait
+// there, rotate, write Z(i) into buffer s and arrive on ZFULL[s]; the quant
+// warps wait there, quantize Z(i) and only then load X(i + 2) into the same
+// buffer.  Hand-offs are named barriers (bar.arrive by the producer,
+// bar.sync by the consumer), which order the shared-memory accesses of both
+// sides; every barrier use alternates with the opposite one, so no
+// generation is ever skipped.  The input of tile i + 2 is fetched into
+// registers before the quant warps wait for Z(i), so its global-memory
+// latency overlaps the MMA stages.
+//
+// Shared memory: P2T [b][b+4] and P1T [a][a+4] (float64), YT [R][b][a+4]
+// (float64, MMA warps only), and two X/Z buffers of R*a rows x (b+4) floats.
+// ---------------------------------------------------------------------------
+constexpr int kWsMmaWarps = 8;
+constexpr int kWsQWarps = 4;
+constexpr int kWsMmaThreads = 32 * kWsMmaWarps;
+constexpr int kWsQThreads = 32 * kWsQWarps;
+constexpr int kWsThreads = kWsMmaThreads + kWsQThreads;
+constexpr int kWsLoadU = 8;  // input chunks (8 elements) per quant thread in flight
+constexpr size_t kWsSmemLimit = 226u * 1024u;  // dynamic shared memory of one block
+// named barrier ids (0 is __syncthreads)
+constexpr int kBarWsMma = 1;    // MMA warps among themselves
+constexpr int kBarWsQ = 2;      // quant warps among themselves
+constexpr int kBarWsXFull = 3;  // + s: X of buffer s staged
+constexpr int kBarWsZFull = 5;  // + s: Z of buffer s written
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+struct WsLayout {
+  int a, b, R, lda, ldb, ldz;
+  size_t off_p1t, off_yt, off_x, xz_floats, bytes;  // double offsets; floats per X/Z buffer
+};
+
+__host__ __device__ inline WsLayout ws_layout(int a, int b, int R) {
+  WsLayout L;
+  L.a = a;
+  L.b = b;
+  L.R = R;
+  L.lda = a + 4;
+  L.ldb = b + 4;
+  L.ldz = b + 4;
+  L.off_p1t = (size_t)b * L.ldb;
+  L.off_yt = L.off_p1t + (size_t)a * L.lda;
+  L.off_x = L.off_yt + (size_t)R * b * L.lda;
+  L.xz_floats = (size_t)R * a * L.ldb;
+  L.bytes = 8 * L.off_x + 4 * 2 * L.xz_floats;
+  return L;
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
+    const Tin* __restrict__ x, int64_t M, int K, const float* __restrict__ P1, int a,
+    const float* __restrict__ P2, int b, int R, const LoopSegs segs, int qmax,
+    int8_t* __restrict__ codes8, int opf, uint8_t* __restrict__ codes4,
+    float* __restrict__ scales, int x_early) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  if (!x_early) pdl_wait();
+  const WsLayout L = ws_layout(a, b, R);
+  double* sm = reinterpret_cast<double*>(smem_raw);
+  double* P2T = sm;
+  double* P1T = sm + L.off_p1t;
+  double* YT = sm + L.off_yt;
+  float* XZ0 = reinterpret_cast<float*>(sm + L.off_x);
+  __shared__ float row_c[2][16];  // clip of each row of each buffer
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int row_chunks = K >> 3;
+  const FastDiv fd_rowc((uint32_t)row_chunks), fd_b((uint32_t)b), fd_a((uint32_t)a);
+
+  // factors, all threads, float64, transposed
+  {
+    constexpr int kFU = 16;
+    const int n2 = b * b, nf = n2 + a * a;
+    for (int base = 0; base < nf; base += kFU * kWsThreads) {
+      float v[kFU];
+#pragma unroll
+      for (int u = 0; u < kFU; ++u) {
+        const int e = base + u * kWsThreads + tid;
+        v[u] = e < n2 ? __ldg(P2 + e) : (e < nf ? __ldg(P1 + (e - n2)) : 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kFU; ++u) {
+        const int e = base + u * kWsThreads + tid;
+        if (e < n2) {  // P2T[j][q] = P2[q][j]
+          const int q = (int)fd_b.div((uint32_t)e), j = e - q * b;
+          P2T[(size_t)j * L.ldb + q] = (double)v[u];
+        } else if (e < nf) {  // P1T[i][p] = P1[p][i]
+          const int e1 = e - n2, p = (int)fd_a.div((uint32_t)e1), i = e1 - p * a;
+          P1T[(size_t)i * L.lda + p] = (double)v[u];
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  const int64_t n_tiles = (M + R - 1) / R;
+  const int64_t my_tiles =
+      n_tiles > (int64_t)blockIdx.x ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (warp < kWsMmaWarps) {
+    // ---------------- MMA warps ----------------
+    const int ct = b >> 3;
+    const int s1_ctq = (ct + kRotTN - 1) / kRotTN;
+    const int s1_tasks = ((R * a) / (8 * kRotTM)) * s1_ctq;
+    const int s2_rt = a / (8 * kRotTM);
+    const int s2_tasks = R * s2_rt * s1_ctq;
+    const FastDiv fd_s1ctq((uint32_t)s1_ctq), fd_s2tok((uint32_t)(s2_rt * s1_ctq));
+    for (int64_t it = 0; it < my_tiles; ++it) {
+      const int sb = (int)(it & 1);
+      float* XZ = XZ0 + sb * L.xz_floats;
+      named_sync(kBarWsXFull + sb, kWsThreads);  // X(it) staged
+      // stage 1: Y[(r,i), j] = sum_q X[(r,i), q] P2[q, j]  -> YT[r][j][i]
+      for (int task = warp; task < s1_tasks; task += kWsMmaWarps) {
+        const int rt = (int)fd_s1ctq.div((uint32_t)task), cq = task - rt * s1_ctq;
+        warp_mma_task<kRotTM, kRotTN>(XZ, L.ldb, P2T, L.ldb, b, rt * 8 * kRotTM, cq * kRotTN, ct,
+                                      [&](int ri, int j, double v0, double v1) {
+                                        const int r = (int)fd_a.div((uint32_t)ri), i = ri - r * a;
+                                        double* yt = YT + ((size_t)r * b + j) * L.lda + i;
+                                        yt[0] = v0;
+                                        yt[L.lda] = v1;
+                                      });
+      }
+      named_sync(kBarWsMma, kWsMmaThreads);  // YT complete, X(it) no longer read
+      // stage 2: Z[r][i][j] = sum_p P1[p, i] Y[r][p][j], rounded once to float32
+      for (int task = warp; task < s2_tasks; task += kWsMmaWarps) {
+        const int r = (int)fd_s2tok.div((uint32_t)task);
+        const int rem = task - r * (s2_rt * s1_ctq);
+        const int rt = (int)fd_s1ctq.div((uint32_t)rem), cq = rem - rt * s1_ctq;
+        warp_mma_task<kRotTM, kRotTN>(P1T, L.lda, YT + (size_t)r * b * L.lda, L.lda, a,
+                                      rt * 8 * kRotTM, cq * kRotTN, ct,
+                                      [&](int i, int j, double v0, double v1) {
+                                        float2* z = reinterpret_cast<float2*>(
+                                            XZ + (size_t)(r * a + i) * L.ldz + j);
+                                        *z = make_float2(__double2float_rn(v0),
+                                                         __double2float_rn(v1));
+                                      });
+      }
+      named_arrive(kBarWsZFull + sb, kWsThreads);  // Z(it) written
+      named_sync(kBarWsMma, kWsMmaThreads);        // YT free for the next tile
+    }
+  } else {
+    // ---------------- quant warps: stage inputs, quantize outputs ----------------
+    const int qt = tid - kWsMmaThreads;
+    const int n_chunks = R * row_chunks;
+    bool waited = !x_early;
+    RawChunk<Tin> xr[kWsLoadU];
+    // load the input of tile `it` into registers (first kWsLoadU chunks per thread)
+    auto fetch = [&](int64_t it) {
+      const int64_t m0 = ((int64_t)blockIdx.x + it * gridDim.x) * R;
+#pragma unroll
+      for (int u = 0; u < kWsLoadU; ++u) {
+        const int ch = u * kWsQThreads + qt;
+        const int r = (int)fd_rowc.div((uint32_t)ch);
+        if (ch < n_chunks && m0 + r < M) {
+          const int64_t gr = m0 + r, j = gr / segs.seg_rows;
+          xr[u].load(x + j * segs.x_stride + (gr - j * segs.seg_rows) * K, ch - r * row_chunks);
+        } else {
+          xr[u].zero();
+        }
+      }
+    };
+    // store tile `it`'s input into its buffer (the registers, then any rest directly)
+    auto stage = [&](int64_t it) {
+      const int sb = (int)(it & 1);
+      float* X = XZ0 + sb * L.xz_floats;
+      const int64_t m0 = ((int64_t)blockIdx.x + it * gridDim.x) * R;
+#pragma unroll
+      for (int u = 0; u < kWsLoadU; ++u) {
+        const int ch = u * kWsQThreads + qt;
+        if (ch < n_chunks) {
+          const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
+          const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
+          xr[u].store(X + (size_t)(r * a + i) * L.ldb + q);
+        }
+      }
+      for (int ch = kWsLoadU * kWsQThreads + qt; ch < n_chunks; ch += kWsQThreads) {
+        const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
+        const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
+        RawChunk<Tin> v;
+        if (m0 + r < M) {
+          const int64_t gr = m0 + r, j = gr / segs.seg_rows;
+          v.load(x + j * segs.x_stride + (gr - j * segs.seg_rows) * K, ch - r * row_chunks);
+        } else {
+          v.zero();
+        }
+        v.store(X + (size_t)(r * a + i) * L.ldb + q);
+      }
+      if (qt < R) {
+        const int64_t gr = m0 + qt, j = gr / segs.seg_rows;
+        float cj = segs.c[0];  // static indices keep the parameter block out of local memory
+#pragma unroll
+        for (int u = 1; u < kMaxLoopsPerLaunch; ++u)
+          if (j == u) cj = segs.c[u];
+        row_c[sb][qt] = cj;
+      }
+    };
+    for (int64_t it = 0; it < my_tiles + 2; ++it) {
+      const int sb = (int)(it & 1);
+      if (it < my_tiles) fetch(it);
+      if (it >= 2) {
+        // quantize Z(it - 2) from buffer sb
+        named_sync(kBarWsZFull + sb, kWsThreads);
+        if (!waited) {  // the previous kernel may still read the output buffers
+          pdl_wait();
+          waited = true;
+        }
+        const float* Z = XZ0 + sb * L.xz_floats;
+        const int64_t m0 = ((int64_t)blockIdx.x + (it - 2) * gridDim.x) * R;
+        const int rows = (M - m0 < (int64_t)R) ? (int)(M - m0) : R;
+        for (int base = 0; base < n_chunks; base += kWsQThreads) {
+          const int ch = base + qt;
+          const int r = (int)fd_rowc.div((uint32_t)ch);
+          const bool valid = ch < n_chunks && r < rows;
+          float v[8];
+          const float c = valid ? row_c[sb][r] : 1.f;
+          if (valid) {
+            const int k8 = (ch - r * row_chunks) * 8;
+            const int i = (int)fd_b.div((uint32_t)k8), j = k8 - i * b;
+            const float4* src = reinterpret_cast<const float4*>(Z + (size_t)(r * a + i) * L.ldz + j);
+            const float4 u0 = src[0], u1 = src[1];
+            v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+            v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+          }
+          uint32_t q[8];
+          const float sc = quant_group8(v, c, qmax, q);
+          if (valid) store_codes<false>(q, sc, m0 * row_chunks + ch, codes8, opf, codes4, scales);
+        }
+        named_sync(kBarWsQ, kWsQThreads);  // Z(it - 2) and its clips fully read
+      }
+      if (it < my_tiles) {
+        stage(it);
+        named_arrive(kBarWsXFull + sb, kWsThreads);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // fused rotation + quantization for a few token rows (decode)
 //
 // With only a handful of rows the row-tile kernel above leaves most SMs idle
@@ -805,6 +1062,31 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
     if ((e = set_smem(k, ssm)) != cudaSuccess) return e;
     return launch_kernel(k, dim3(grid), dim3(kThreads), ssm, s, pdl, (const float*)x, (int)K,
                          P1, a, P2, b, segs, qmax, codes8, opf, codes4, scales, asum, xe);
+  }
+  {  // many rows: the warp-specialised kernel, one persistent block per SM
+    int Rw = 0;
+    for (int r = 16; r >= 1; r >>= 1)
+      if (ws_layout(a, b, r).bytes <= kWsSmemLimit) {
+        Rw = r;
+        break;
+      }
+    if (Rw > 0 && opf != kOpGemvAct && M >= (int64_t)Rw * num_sms() * 4) {
+      const size_t wsm = ws_layout(a, b, Rw).bytes;
+      const int64_t tiles = (M + Rw - 1) / Rw;
+      const int grid = (int)std::min<int64_t>(tiles, (int64_t)num_sms());
+      cudaError_t e;
+      if (x_dtype == LQ_BF16) {
+        auto* k = k_rotate_quant_ws<__nv_bfloat16>;
+        if ((e = set_smem(k, wsm)) != cudaSuccess) return e;
+        return launch_kernel(k, dim3(grid), dim3(kWsThreads), wsm, s, pdl,
+                             (const __nv_bfloat16*)x, M, (int)K, P1, a, P2, b, Rw, segs, qmax,
+                             codes8, opf, codes4, scales, xe);
+      }
+      auto* k = k_rotate_quant_ws<float>;
+      if ((e = set_smem(k, wsm)) != cudaSuccess) return e;
+      return launch_kernel(k, dim3(grid), dim3(kWsThreads), wsm, s, pdl, (const float*)x, M,
+                           (int)K, P1, a, P2, b, Rw, segs, qmax, codes8, opf, codes4, scales, xe);
+    }
   }
   int R = 0;
   size_t smem = rotate_smem_bytes(a, b, &R);

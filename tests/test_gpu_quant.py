@@ -118,6 +118,32 @@ def test_fused_rotate_quantize_few_rows(M, ab, x_dtype):
             np.testing.assert_array_equal(O.unpack_int4(host(q4)), host(q8))
 
 
+@pytest.mark.parametrize("ab,M", [((32, 64), 2368 + 37), ((64, 88), 592 + 5), ((16, 16), 9472 + 301),
+                                  ((16, 128), 2368 * 2 + 1), ((64, 64), 1184 + 129)])
+@pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
+def test_fused_rotate_quantize_many_rows(ab, M, x_dtype):
+    """Enough rows for the warp-specialised kernel (one persistent block per
+    SM, at least four row tiles per block; tiles of 16, 4 or 1 rows by factor
+    size), with a ragged last tile and blocks holding one tile more than
+    others: every code against the oracle (only near-tie differences)."""
+    a, b = ab
+    K = a * b
+    x = _outlier_matrix(M, K, seed=M + K)
+    if x_dtype == "bf16":
+        x = synth.round_bf16(x)
+    P1, P2 = _orthogonal(a, a + 5), _orthogonal(b, b + 6)
+    xt64 = O.kron_rotate_f64(x, P1, P2)
+    for bits in (4, 8):
+        q8, q4, s = lq.lq_quantize_act(act_tensor(x, x_dtype), dev(P1), dev(P2), 0.91, bits,
+                                       want_codes4=(bits == 4))
+        torch.cuda.synchronize()
+        q_or, s_or = O.quantize_groups(xt64.astype(np.float32), 0.91, bits)
+        flips = check_codes_near_tie(host(q8), host(s), q_or, s_or, xt64)
+        assert len(flips) == 0
+        if bits == 4:
+            np.testing.assert_array_equal(O.unpack_int4(host(q4)), host(q8))
+
+
 def test_fused_rotation_identity_factors_reduce_to_plain_rtn():
     M, K = 100, 2048
     x = _outlier_matrix(M, K, seed=3)
