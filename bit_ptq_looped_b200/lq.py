@@ -16,7 +16,9 @@ import numpy as np
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "liblq.so")
+# LQ_LIB_PATH selects another build of the same library (the host-sanitizer
+# build in the sanitizer test); by default the in-tree liblq.so
+LIB_PATH = os.environ.get("LQ_LIB_PATH") or os.path.join(HERE, "liblq.so")
 
 LQ_OK, LQ_ERR_ARG, LQ_ERR_SHAPE, LQ_ERR_UNSUPPORTED, LQ_ERR_ALIGN = 0, 1, 2, 3, 4
 LQ_ERR_CUDA, LQ_ERR_DEVICE_TIMEOUT, LQ_ERR_NOMEM, LQ_ERR_WORKSPACE = 5, 6, 7, 8
