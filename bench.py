@@ -623,6 +623,115 @@ def measure_stack(lq, ctx, wl, n_steps, warmup, n_probe, peaks, want_clocks=Fals
     return line, (layers, packed, x, y, ws, copies)
 
 
+def aux_schedules(lq, ctx, wl, layers, x_dev, ops_step):
+    """The same step under other schedules of the loop driver: loop by loop
+    (workspace for one loop), and SLT serving with every module selected (its
+    own transform and weight at every loop, so no loop shares a launch)."""
+    torch, dev, stream, timed = ctx.torch, ctx.dev, ctx.stream, ctx.timed
+    params = synth.module_params(wl)
+    out = {}
+    M, T, L = wl.M, wl.T, len(wl.linears)
+    y = torch.empty(T * M * sum(lin.N for lin in wl.linears), dtype=torch.float32, device=dev)
+    n = 50
+
+    ws1 = lq.workspace(layers, M, dev)
+    run = lambda: lq.lq_loop_stack(x_dev, layers, T, lq.LQ_OPEN, M=M, y=y, ws=ws1,
+                                   stream=stream)
+    for _ in range(3):
+        run()
+    ms = timed(n, run) / n
+    out["loop_by_loop"] = {"ms_per_step": ms, "TOPS": ops_step / (ms * 1e-3) / 1e12,
+                           "launches_per_step": 2 * T * L}
+
+    lins = wl.linears
+    if all(lins[l].N == lins[(l + 1) % L].K for l in range(L)):
+        # chain mode: loops strictly in sequence, y of each step feeding the next
+        # (inputs: the first step's x), plain and with CTA at the T - 1 transitions
+        x0 = x_dev[: M * lins[0].K]
+        run = lambda: lq.lq_loop_stack(x0, layers, T, lq.LQ_CHAIN, M=M, y=y, ws=ws1,
+                                       stream=stream)
+        for _ in range(3):
+            run()
+        ms = timed(n, run) / n
+        out["chain"] = {"ms_per_step": ms, "TOPS": ops_step / (ms * 1e-3) / 1e12}
+        d = lins[-1].N
+        rng = np.random.default_rng(23)
+        U = torch.from_numpy((0.05 * rng.standard_normal((d, 8))).astype(np.float32)).to(dev)
+        V = torch.from_numpy((0.05 * rng.standard_normal((d, 8))).astype(np.float32)).to(dev)
+        a = torch.from_numpy((1 + 0.1 * rng.standard_normal((T - 1, d))).astype(np.float32)).to(dev)
+        b = torch.from_numpy((0.1 * rng.standard_normal((T - 1, d))).astype(np.float32)).to(dev)
+        cta = lq.lq_cta_create(U, V, a, b, rng.uniform(0.1, 0.9, T - 1))
+        ws_c = torch.empty(lq.lq_cta_stack_workspace_bytes(layers, M), dtype=torch.uint8,
+                           device=dev)
+        run = lambda: lq.lq_loop_stack_cta(x0, layers, T, cta, M=M, y=y, ws=ws_c, stream=stream)
+        for _ in range(3):
+            run()
+        ms_c = timed(n, run) / n
+        out["chain_cta"] = {"ms_per_step": ms_c, "TOPS": ops_step / (ms_c * 1e-3) / 1e12,
+                            "transitions": T - 1,
+                            "us_per_transition": (ms_c - ms) * 1e3 / max(T - 1, 1)}
+        cta.free()
+
+    # trajectory Hessian of the first module over its T loop inputs (bf16)
+    lin0 = lins[0]
+    if wl.x_dtype == "bf16" and lin0.K % 128 == 0:
+        K0 = lin0.K
+        xh = torch.empty(T * M * K0, dtype=torch.bfloat16, device=dev)
+        off = 0
+        for t in range(T):  # loop t's input of module 0 inside the open-mode buffer
+            src = x_dev[(t * sum(l.K for l in lins)) * M: (t * sum(l.K for l in lins) + K0) * M]
+            xh[off: off + M * K0] = src
+            off += M * K0
+        Hh = torch.empty((K0, K0), dtype=torch.float32, device=dev)
+        wsh = torch.empty(lq.lib().lq_hessian_workspace_bytes(M, K0, T), dtype=torch.uint8,
+                          device=dev)
+        run = lambda: lq.lq_trajectory_hessian(xh, T, M=M, H=Hh, ws=wsh, stream=stream)
+        for _ in range(3):
+            run()
+        ms_h = timed(n, run) / n
+        flops = T * M * K0 * (K0 + 1)  # the symmetric product: one multiply-add per pair i <= j
+        peaks = load_peaks()
+        out["trajectory_hessian"] = {
+            "workload": f"H = sum_t X_t^T X_t, T={T} x {M} x {K0} bf16 -> {K0}x{K0} fp32",
+            "us": ms_h * 1e3, "TFLOP_s": flops / (ms_h * 1e-3) / 1e12,
+            "frac_bf16_peak": flops / (ms_h * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "flops": flops, "includes": "bf16 transpose of the inputs (one launch) + the product"}
+        del xh, Hh, wsh
+
+    rng = np.random.default_rng(17)
+    own, keep = [], []
+    for t in range(T):
+        row = []
+        for mp in params:
+            a, b = mp.P1.shape[0], mp.P2.shape[0]
+            P1 = np.linalg.qr(rng.standard_normal((a, a)))[0].astype(np.float32)
+            P2 = np.linalg.qr(rng.standard_normal((b, b)))[0].astype(np.float32)
+            Q1 = lq.lq_inverse_transpose(P1).to(dev)
+            Q2 = lq.lq_inverse_transpose(P2).to(dev)
+            Wf = lq.lq_fold_weights(torch.from_numpy(mp.W).to(dev), Q1, Q2)
+            wq = lq.lq_pack_weights(Wf)
+            del Wf
+            row.append(lq.lq_layer_create(wq, torch.from_numpy(P1).to(dev),
+                                          torch.from_numpy(P2).to(dev), mp.las, wl.a_bits))
+            keep.append(wq)
+        own.append(row)
+    ws2 = lq.workspace(layers, M, dev, T=T)
+    run = lambda: lq.lq_loop_stack_slt(x_dev, own, lq.LQ_OPEN, M=M, y=y, ws=ws2, stream=stream)
+    for _ in range(3):
+        run()
+    ms = timed(n, run) / n
+    shared_bytes = sum(l.wq.info()["device_bytes"] for l in layers)
+    out["slt_all_selected"] = {"ms_per_step": ms, "TOPS": ops_step / (ms * 1e-3) / 1e12,
+                               "resident_weight_bytes": T * shared_bytes,
+                               "shared_weight_bytes": shared_bytes}
+    for row in own:
+        for l in row:
+            l.free()
+    for wq in keep:
+        wq.free()
+    return out
+
+
 def aux_hbm_kernels(lq, ctx, peaks):
     """The quantize-only kernel and the streaming GEMV on launches far larger than L2."""
     torch, dev, stream = ctx.torch, ctx.dev, ctx.stream
@@ -727,6 +836,12 @@ def run_lq(args, rank, world, local_rank):
             awl = WORKLOADS[name]
             steps = 10 if is_decode(awl) else 100
             a_line, a_held = measure_stack(lq, ctx, awl, steps, 3, steps, peaks)
+            if name == synth.ATTN_PROJ.name:
+                # the same linear under the driver's other schedules (loop by
+                # loop, chain, chain with loop-transition adapters, SLT serving)
+                # and the trajectory Hessian of its loop inputs
+                a_line["schedules"] = aux_schedules(lq, ctx, awl, a_held[0], a_held[2],
+                                                    work_per_step(awl)[0])
             free_layers(a_held[0], a_held[1])
             del a_held
             aux[name] = a_line

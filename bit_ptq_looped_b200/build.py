@@ -14,6 +14,8 @@ LIB = os.path.join(HERE, "liblq.so")
 # the C++ of the library; the device code is unchanged), loaded instead of
 # liblq.so when LQ_LIB_PATH points at it
 LIB_SAN = os.path.join(HERE, "liblq_san.so")
+# bounds-check build: kernels test their store indices and record violations
+LIB_BOUNDS = os.path.join(HERE, "liblq_bounds.so")
 SAN_FLAGS = ["-Xcompiler", "-fsanitize=address,-fsanitize=undefined,-fno-omit-frame-pointer,-g",
              "-lasan", "-lubsan"]
 SOURCES = ["lq_api.cu", "lq_quant.cu", "lq_gemm.cu", "lq_gemv.cu", "lq_cta.cu", "lq_noalloc.cu"]
@@ -55,6 +57,11 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None, lib: str
 def build_sanitized(force: bool = False) -> str:
     """liblq_san.so: the same sources with the host code under ASan + UBSan."""
     return build(force=force, extra_flags=SAN_FLAGS, lib=LIB_SAN)
+
+
+def build_bounds_checked(force: bool = False) -> str:
+    """liblq_bounds.so: the kernels test their store indices (-DLQ_BOUNDS_CHECK)."""
+    return build(force=force, extra_flags=["-DLQ_BOUNDS_CHECK"], lib=LIB_BOUNDS)
 
 
 if __name__ == "__main__":

@@ -35,12 +35,14 @@ lq_status cuda_error(cudaError_t e, const char* what) {
 
 using namespace lq;
 
+// Resident weights: only the packed 4-bit codes and their float32 steps.  The
+// tensor-core GEMM reads an 8-bit operand copy (E4M3 or int8 bytes) and the
+// steps transposed (G x N); both are expanded into the caller's workspace by
+// each call that runs the GEMM (once per launch, which covers up to 8 loops).
 struct lq_wq {
   int64_t N = 0, K = 0, G = 0;
   uint8_t* codes4 = nullptr;   // N x K/2 packed
   float* scales = nullptr;     // N x G
-  float* scales_t = nullptr;   // G x N (tensor-core GEMM layout)
-  uint8_t* op[2] = {nullptr, nullptr};  // N x K operand copies: [kOpInt8], [kOpE4M3]
   int device = 0;
   int64_t bytes = 0;
 };
@@ -145,6 +147,18 @@ int64_t ws_bytes_for(int64_t M, int64_t K) {
   return round_up(M * K, 256) + steps + (use_gemv(M, K) ? steps : 0);
 }
 
+// the GEMM's weight operand in the workspace: N x K code bytes, then the
+// steps transposed (G x N float32)
+int64_t op_bytes_for(int64_t N, int64_t K) {
+  return round_up(N * K, 256) + round_up(N * (K / kGroup) * 4, 256);
+}
+
+// workspace of one linear call: activation codes and steps, plus the weight
+// operand when the call takes the tensor-core path
+int64_t ws_bytes_linear(int64_t M, int64_t K, int64_t N) {
+  return round_up(ws_bytes_for(M, K), 256) + (use_gemv(M, K) ? 0 : op_bytes_for(N, K));
+}
+
 // Graph cache of the loop driver: one instantiated graph per argument set.
 struct GraphKey {
   const void* x;
@@ -218,7 +232,13 @@ struct Probe {
 };
 Probe g_probe;
 
-enum ProbeKind { kProbeRotQuant = 0, kProbeQuant = 1, kProbeGemm = 2, kProbeGemv = 3 };
+enum ProbeKind {
+  kProbeRotQuant = 0,
+  kProbeQuant = 1,
+  kProbeGemm = 2,
+  kProbeGemv = 3,
+  kProbeWeightOp = 4
+};
 
 struct ProbeScope {
   cudaEvent_t a = nullptr, b = nullptr;
@@ -287,9 +307,17 @@ lq_status enqueue_linear(const void* x, int32_t x_dtype, int64_t M, const lq_lay
                           s, pdl);
     if (e != cudaSuccess) return cuda_error(e, "gemv launch");
   } else {
+    // the weight operand for this launch, expanded from the resident 4-bit codes
+    uint8_t* op = (uint8_t*)ws + round_up(ws_bytes_for(Mt, K), 256);
+    float* sw_t = (float*)(op + round_up(N * K, 256));
+    {
+      ProbeScope pw(kProbeWeightOp, s);
+      e = launch_weight_operand(wq->codes4, wq->scales, N, K, opf, op, sw_t, s, pdl);
+    }
+    if (e != cudaSuccess) return cuda_error(e, "weight operand launch");
     ProbeScope ps(kProbeGemm, s);
     const char* why = nullptr;
-    e = launch_group_gemm(codes, scales, wq->op[opf], wq->scales_t, y, Mt, N, K, opf, s, &why,
+    e = launch_group_gemm(codes, scales, op, sw_t, y, Mt, N, K, opf, s, &why,
                           pdl, nb > 1 ? M : INT64_MAX, y_stride);
     if (e != cudaSuccess) {
       if (why) {
@@ -308,9 +336,51 @@ int loops_per_launch(const lq_layer* L, int64_t M, int T, int64_t ws_bytes) {
   const int64_t K = L->wq->K;
   if (use_gemv(M, K) || L->P1 == nullptr) return 1;
   int nb = std::min(T, kMaxLoopsPerLaunch);
-  while (nb > 1 && (ws_bytes_for(M * nb, K) > ws_bytes || M * nb > ((int64_t)1 << 31) - 256))
+  while (nb > 1 && (ws_bytes_linear(M * nb, K, L->wq->N) > ws_bytes ||
+                    M * nb > ((int64_t)1 << 31) - 256))
     --nb;
   return nb;
+}
+
+// Decode-sized open-mode stacks: the (t, l) steps are independent, so they
+// run as kDecodeBranches concurrent chains (quantize, then GEMV, each chain
+// with its own slice of the workspace), forked from and joined back into the
+// caller's stream.  Per device: the branch streams and the fork/join events.
+constexpr int kDecodeBranches = 16;
+struct BranchSet {
+  cudaStream_t st[kDecodeBranches];
+  cudaEvent_t fork;
+  cudaEvent_t join[kDecodeBranches];
+};
+std::mutex g_branch_mu;
+std::map<int, BranchSet> g_branch_sets;
+
+lq_status branch_set(BranchSet** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+  auto it = g_branch_sets.find(dev);
+  if (it == g_branch_sets.end()) {
+    BranchSet b{};
+    for (int i = 0; i < kDecodeBranches; ++i) {
+      if ((e = cudaStreamCreateWithFlags(&b.st[i], cudaStreamNonBlocking)) != cudaSuccess)
+        return cuda_error(e, "create branch stream");
+      if ((e = cudaEventCreateWithFlags(&b.join[i], cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_error(e, "create branch event");
+    }
+    if ((e = cudaEventCreateWithFlags(&b.fork, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_error(e, "create branch event");
+    it = g_branch_sets.emplace(dev, b).first;
+  }
+  *out = &it->second;
+  return LQ_OK;
+}
+
+// workspace slice of one decode branch (the largest layer's codes, steps and sums)
+int64_t decode_branch_bytes(const std::vector<const lq_layer*>& tl, int64_t M) {
+  int64_t per = 0;
+  for (const lq_layer* ly : tl) per = std::max(per, round_up(ws_bytes_for(M, ly->wq->K), 256));
+  return per;
 }
 
 lq_status check_layer_call(const lq_layer* layer, int64_t M, int32_t x_dtype) {
@@ -327,10 +397,6 @@ lq_status check_layer_call(const lq_layer* layer, int64_t M, int32_t x_dtype) {
     return LQ_ERR_ARG;
   }
   const bool gemm = !use_gemv(M, layer->wq->K);
-  if (gemm && layer->wq->op[layer->a_bits == 4 ? kOpE4M3 : kOpInt8] == nullptr) {
-    set_error("layer has no tensor-core operand copy");
-    return LQ_ERR_ARG;
-  }
   if (gemm && layer->wq->K % 128) {
     set_error("K=%lld must be a multiple of 128 for the tensor-core path (M > %d)",
               (long long)layer->wq->K, kGemvMaxM);
@@ -510,16 +576,14 @@ lq_status lq_pack_weights(const float* d_W_folded, int64_t N, int64_t K, int32_t
   cudaError_t e;
   const size_t b4 = (size_t)N * K / 2, bs = (size_t)N * w->G * 4;
   if ((e = cudaMalloc(&w->codes4, b4)) != cudaSuccess ||
-      (e = cudaMalloc(&w->scales, bs)) != cudaSuccess ||
-      (e = cudaMalloc(&w->scales_t, bs)) != cudaSuccess) {
+      (e = cudaMalloc(&w->scales, bs)) != cudaSuccess) {
     lq_wq_free(w);
-    set_error("cudaMalloc of %zu bytes failed: %s", b4 + 2 * bs, cudaGetErrorString(e));
+    set_error("cudaMalloc of %zu bytes failed: %s", b4 + bs, cudaGetErrorString(e));
     return LQ_ERR_NOMEM;
   }
-  w->bytes = (int64_t)(b4 + 2 * bs);
+  w->bytes = (int64_t)(b4 + bs);
   e = launch_quantize(d_W_folded, LQ_F32, N, K, nullptr, 0, nullptr, 0, one_loop(1.0f), 4,
                       nullptr, kOpInt8, w->codes4, w->scales, s);
-  if (e == cudaSuccess) e = launch_transpose_f32(w->scales, N, w->G, w->scales_t, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     lq_wq_free(w);
@@ -547,9 +611,7 @@ void lq_wq_free(lq_wq* wq) {
   if (!wq) return;
   cudaFree(wq->codes4);
   cudaFree(wq->scales);
-  cudaFree(wq->scales_t);
-  cudaFree(wq->op[0]);
-  cudaFree(wq->op[1]);
+
   delete wq;
 }
 
@@ -596,26 +658,6 @@ lq_status lq_layer_create(const lq_wq* wq, const float* d_P1, int32_t a, const f
     lq_layer_free(L);
     return cuda_error(e, "copy Kronecker factors");
   }
-  // tensor-core operand copy of the weight codes (int8 for W4A8, E4M3 for W4A4)
-  const int opf = a_bits == 4 ? kOpE4M3 : kOpInt8;
-  lq_wq* w = const_cast<lq_wq*>(wq);
-  if (w->op[opf] == nullptr) {
-    uint8_t* buf = nullptr;
-    if ((e = cudaMalloc(&buf, (size_t)w->N * w->K)) != cudaSuccess) {
-      lq_layer_free(L);
-      set_error("cudaMalloc of the operand copy failed: %s", cudaGetErrorString(e));
-      return LQ_ERR_NOMEM;
-    }
-    e = launch_codes4_to_operand(w->codes4, w->N * w->K / 2, opf, buf, 0);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
-    if (e != cudaSuccess) {
-      cudaFree(buf);
-      lq_layer_free(L);
-      return cuda_error(e, "operand copy");
-    }
-    w->op[opf] = buf;
-    w->bytes += w->N * w->K;
-  }
   *out = L;
   return LQ_OK;
 }
@@ -633,7 +675,7 @@ int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M) 
   int64_t need = 0;
   for (int i = 0; i < L; ++i) {
     if (!layers[i]) return -1;
-    need = std::max(need, ws_bytes_for(M, layers[i]->wq->K));
+    need = std::max(need, ws_bytes_linear(M, layers[i]->wq->K, layers[i]->wq->N));
   }
   return need;
 }
@@ -647,7 +689,14 @@ int64_t lq_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64
     const int64_t K = layers[i]->wq->K;
     const bool batch = !use_gemv(M, K) && layers[i]->P1 != nullptr;
     const int nb = batch ? std::min<int>(T, kMaxLoopsPerLaunch) : 1;
-    need = std::max(need, ws_bytes_for(M * nb, K));
+    need = std::max(need, ws_bytes_linear(M * nb, K, layers[i]->wq->N));
+  }
+  bool decode = (int64_t)T * L > 1;
+  for (int i = 0; i < L; ++i) decode = decode && use_gemv(M, layers[i]->wq->K);
+  if (decode) {  // one workspace slice per concurrent decode chain
+    const std::vector<const lq_layer*> tl(layers, layers + L);
+    need = std::max(need, decode_branch_bytes(tl, M) *
+                              std::min<int64_t>(kDecodeBranches, (int64_t)T * L));
   }
   return need;
 }
@@ -669,9 +718,9 @@ lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_l
     set_error("x and y must be 16-byte aligned and the workspace 256-byte aligned");
     return LQ_ERR_ALIGN;
   }
-  if (ws_bytes < ws_bytes_for(M, layer->wq->K)) {
+  if (ws_bytes < ws_bytes_linear(M, layer->wq->K, layer->wq->N)) {
     set_error("workspace of %lld bytes is smaller than the %lld needed", (long long)ws_bytes,
-              (long long)ws_bytes_for(M, layer->wq->K));
+              (long long)ws_bytes_linear(M, layer->wq->K, layer->wq->N));
     return LQ_ERR_WORKSPACE;
   }
   return enqueue_linear(d_x, x_dtype, M, layer, t, d_y, d_ws, (cudaStream_t)stream);
@@ -692,6 +741,46 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
     for (int l = 0; l < L; ++l) {
       sum_k += at(0, l)->wq->K;
       sum_n += at(0, l)->wq->N;
+    }
+    bool decode = T * L > 1;
+    for (const lq_layer* ly : tl) decode = decode && use_gemv(M, ly->wq->K);
+    if (decode) {
+      const int64_t per = decode_branch_bytes(tl, M);
+      const int nbr = (int)std::min(std::min((int64_t)kDecodeBranches, (int64_t)T * L),
+                                    ws_bytes / per);
+      if (nbr >= 2) {
+        std::lock_guard<std::mutex> lk(g_branch_mu);
+        BranchSet* bs = nullptr;
+        lq_status st = branch_set(&bs);
+        if (st != LQ_OK) return st;
+        cudaError_t e = cudaEventRecord(bs->fork, s);
+        if (e != cudaSuccess) return cuda_error(e, "fork record");
+        for (int b = 0; b < nbr; ++b)
+          if ((e = cudaStreamWaitEvent(bs->st[b], bs->fork, 0)) != cudaSuccess)
+            return cuda_error(e, "fork wait");
+        int i = 0;
+        for (int t = 0; t < T && st == LQ_OK; ++t) {
+          int64_t k_before = 0, n_before = 0;
+          for (int l = 0; l < L; ++l, ++i) {
+            const lq_layer* ly = at(t, l);
+            const int b = i % nbr;
+            const char* xin = (const char*)d_x + (size_t)(M * (t * sum_k + k_before)) * esz;
+            float* yout = d_y + M * (t * sum_n + n_before);
+            st = enqueue_linear(xin, x_dtype, M, ly, t, yout, (char*)d_ws + (size_t)b * per,
+                                bs->st[b], i >= nbr, true);
+            if (st != LQ_OK) break;
+            k_before += ly->wq->K;
+            n_before += ly->wq->N;
+          }
+        }
+        // join every branch back (also after an error, so no capture is left unjoined)
+        for (int b = 0; b < nbr; ++b) {
+          cudaError_t e1 = cudaEventRecord(bs->join[b], bs->st[b]);
+          cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(s, bs->join[b], 0) : e1;
+          if (e2 != cudaSuccess && st == LQ_OK) st = cuda_error(e2, "join");
+        }
+        return st;
+      }
     }
     int nb_all = kMaxLoopsPerLaunch;
     for (const lq_layer* ly : tl) nb_all = std::min(nb_all, loops_per_launch(ly, M, T, ws_bytes));
@@ -722,7 +811,8 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
   const float* prev_y = nullptr;
   // CTA state (the adapted input of the next loop) after the codes and steps
   int64_t codes_ws = 0;
-  for (const lq_layer* ly : tl) codes_ws = std::max(codes_ws, ws_bytes_for(M, ly->wq->K));
+  for (const lq_layer* ly : tl)
+    codes_ws = std::max(codes_ws, ws_bytes_linear(M, ly->wq->K, ly->wq->N));
   float* state = (float*)((char*)d_ws + round_up(codes_ws, 256));
   for (int t = 0; t < T; ++t) {
     for (int l = 0; l < L; ++l) {
@@ -774,7 +864,7 @@ static lq_status loop_stack_impl(const void* d_x, int32_t x_dtype, int64_t M,
                   (long long)l0->wq->K);
         return LQ_ERR_SHAPE;
       }
-      need = std::max(need, ws_bytes_for(M, ly->wq->K));
+      need = std::max(need, ws_bytes_linear(M, ly->wq->K, ly->wq->N));
     }
   }
   if (mode == LQ_CHAIN) {
@@ -1142,7 +1232,19 @@ lq_status lq_selftest_bounded_wait(int64_t limit_us, void* stream) {
 lq_status lq_check_device(void* stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_error(e, "pending CUDA error");
-  return read_and_clear_device_status((cudaStream_t)stream);
+  lq_status st = read_and_clear_device_status((cudaStream_t)stream);
+  if (st != LQ_OK) return st;
+  // bounds-check build: an index a kernel found out of range (none otherwise)
+  const char* files[4] = {"lq_quant.cu", "lq_gemm.cu", "lq_gemv.cu", "lq_cta.cu"};
+  const unsigned long long v[4] = {bounds_fail_quant(), bounds_fail_gemm(), bounds_fail_gemv(),
+                                   bounds_fail_cta()};
+  for (int i = 0; i < 4; ++i)
+    if (v[i]) {
+      set_error("index out of range in %s line %llu (index %lld)", files[i], v[i] >> 40,
+                (long long)(v[i] & 0xFFFFFFFFFFull));
+      return LQ_ERR_DEVICE_BOUNDS;
+    }
+  return LQ_OK;
 }
 
 }  // extern "C"
@@ -1175,7 +1277,7 @@ lq_status noalloc_check(const void* d_x, int32_t x_dtype, int64_t M, const lq_la
 }
 
 int64_t noalloc_ws_bytes(const lq_layer* layer, int64_t M) {
-  return ws_bytes_for(M, layer->wq->K);
+  return ws_bytes_linear(M, layer->wq->K, layer->wq->N);
 }
 
 lq_status noalloc_enqueue(const void* d_x, int32_t x_dtype, int64_t M, const lq_layer* layer,

@@ -111,6 +111,41 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 }
 
 // ---------------------------------------------------------------------------
+// Index checks of the bounds-check build (-DLQ_BOUNDS_CHECK).  At the checked
+// stores a kernel tests the index against the extent it writes; an index out
+// of range is recorded (source line and index of the first one, in a status
+// word of the kernel's own source file) and the store is skipped, so the
+// check never writes out of bounds itself.  lq_check_device reports a
+// recorded violation.  In the normal build LQ_IN_RANGE is `true` and costs
+// nothing.
+// ---------------------------------------------------------------------------
+#ifdef LQ_BOUNDS_CHECK
+static __device__ unsigned long long g_lq_bounds_fail = 0ull;
+__device__ __forceinline__ bool lq_in_range(long long idx, long long extent, int line) {
+  if (idx >= 0 && idx < extent) return true;
+  atomicCAS(&g_lq_bounds_fail, 0ull,
+            ((unsigned long long)line << 40) | ((unsigned long long)idx & 0xFFFFFFFFFFull));
+  return false;
+}
+#define LQ_IN_RANGE(idx, extent) lq_in_range((long long)(idx), (long long)(extent), __LINE__)
+// first violation recorded by this source file's kernels (0: none), cleared
+static inline unsigned long long lq_take_bounds_fail() {
+  unsigned long long v = 0ull, z = 0ull;
+  if (cudaMemcpyFromSymbol(&v, g_lq_bounds_fail, sizeof(v)) != cudaSuccess) return ~0ull;
+  if (v) cudaMemcpyToSymbol(g_lq_bounds_fail, &z, sizeof(z));
+  return v;
+}
+#else
+#define LQ_IN_RANGE(idx, extent) true
+static inline unsigned long long lq_take_bounds_fail() { return 0ull; }
+#endif
+// per source file: the first recorded violation of its kernels (0: none)
+unsigned long long bounds_fail_quant();
+unsigned long long bounds_fail_gemm();
+unsigned long long bounds_fail_gemv();
+unsigned long long bounds_fail_cta();
+
+// ---------------------------------------------------------------------------
 // PTX wrappers: mbarrier, TMA, tcgen05
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -326,10 +361,10 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
                             int* asum = nullptr);
 cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const float* Q1, int a,
                                 const float* Q2, int b, float* out, cudaStream_t s);
-cudaError_t launch_codes4_to_operand(const uint8_t* codes4, int64_t n_bytes, int opf,
-                                     uint8_t* out, cudaStream_t s);
-cudaError_t launch_transpose_f32(const float* in, int64_t rows, int64_t cols, float* out,
-                                 cudaStream_t s);
+// The GEMM weight operand of one launch from the resident codes and steps:
+// N x K code bytes (E4M3 or int8 per opf) and the steps transposed to G x N.
+cudaError_t launch_weight_operand(const uint8_t* codes4, const float* sw, int64_t N, int64_t K,
+                                  int opf, uint8_t* op, float* sw_t, cudaStream_t s, bool pdl);
 size_t rotate_smem_bytes(int a, int b, int* rows_per_block);
 
 // GEMM (lq_gemm.cu).  Output row r goes to y + j * y_stride + (r - j * y_seg_rows) * N,

@@ -138,4 +138,6 @@ cudaError_t launch_cta_apply(const float* h, int64_t M, int d, const double* U8,
                        a, b, eta, out);
 }
 
+unsigned long long bounds_fail_cta() { return lq_take_bounds_fail(); }
+
 }  // namespace lq

@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         float* yr = y + jseg * y_stride + (gm - jseg * y_seg_rows) * (int64_t)N + n0 + col0;
 #pragma unroll
         for (int c4 = 0; c4 < EPI_COLS / 4; ++c4) {
-          if (n0 + col0 + 4 * c4 < N)
+          if (n0 + col0 + 4 * c4 < N && LQ_IN_RANGE(n0 + col0 + 4 * c4 + 3, N))
             *reinterpret_cast<float4*>(yr + 4 * c4) =
                 make_float4(acc[2 * c4].x, acc[2 * c4].y, acc[2 * c4 + 1].x, acc[2 * c4 + 1].y);
         }
@@ -744,5 +744,7 @@ lq_status read_and_clear_device_status(cudaStream_t s) {
   }
   return LQ_OK;
 }
+
+unsigned long long bounds_fail_gemm() { return lq_take_bounds_fail(); }
 
 }  // namespace lq

@@ -166,7 +166,9 @@ __global__ void __launch_bounds__(kGemvThreads, kDB ? 1 : 3) k_group_gemv(
       const int n = gw + (j0 + r) * W;
 #pragma unroll
       for (int m = 0; m < MB; ++m)
-        if (lane == ((r * MB + m) & 31) && m < M && n < N) y[(size_t)m * N + n] = part[r][m];
+        if (lane == ((r * MB + m) & 31) && m < M && n < N &&
+            LQ_IN_RANGE((size_t)m * N + n, (size_t)M * N))
+          y[(size_t)m * N + n] = part[r][m];
     }
   };
 
@@ -411,12 +413,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
       for (int j = 0; j < NB; ++j) {
         const int m0 = j * 8 + 2 * t;
         if (na < N) {
-          if (m0 < M) y[(size_t)m0 * N + na] = acc[j][0].x;
-          if (m0 + 1 < M) y[(size_t)(m0 + 1) * N + na] = acc[j][0].y;
+          if (m0 < M && LQ_IN_RANGE(na, N)) y[(size_t)m0 * N + na] = acc[j][0].x;
+          if (m0 + 1 < M && LQ_IN_RANGE(na, N)) y[(size_t)(m0 + 1) * N + na] = acc[j][0].y;
         }
         if (nb < N) {
-          if (m0 < M) y[(size_t)m0 * N + nb] = acc[j][1].x;
-          if (m0 + 1 < M) y[(size_t)(m0 + 1) * N + nb] = acc[j][1].y;
+          if (m0 < M && LQ_IN_RANGE(nb, N)) y[(size_t)m0 * N + nb] = acc[j][1].x;
+          if (m0 + 1 < M && LQ_IN_RANGE(nb, N)) y[(size_t)(m0 + 1) * N + nb] = acc[j][1].y;
         }
         acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
       }
@@ -565,5 +567,7 @@ cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa
     return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
   return launch_tc(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
 }
+
+unsigned long long bounds_fail_gemv() { return lq_take_bounds_fail(); }
 
 }  // namespace lq

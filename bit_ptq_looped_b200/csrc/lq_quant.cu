@@ -435,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
         if (ch < R * row_chunks) {
           const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
           const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
-          xr[u].store(X + (size_t)(r * a + i) * L.ldb + q);
+          const size_t off = (size_t)(r * a + i) * L.ldb + q;
+          if (LQ_IN_RANGE(off + 7, (size_t)R * a * L.ldb)) xr[u].store(X + off);
         }
       }
     } else {
@@ -461,6 +462,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
                                     [&](int ri, int j, double v0, double v1) {
                                       const int r = (int)fd_a.div((uint32_t)ri), i = ri - r * a;
                                       double* yt = YT + ((size_t)r * b + j) * L.lda + i;
+                                      if (!LQ_IN_RANGE(((size_t)r * b + j + 1) * L.lda + i,
+                                                       (size_t)R * b * L.lda))
+                                        return;
                                       yt[0] = v0;
                                       yt[L.lda] = v1;
                                     });
@@ -476,6 +480,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
                                     [&](int i, int j, double v0, double v1) {
                                       float2* z = reinterpret_cast<float2*>(
                                           Z + (size_t)(r * a + i) * L.ldz + j);
+                                      if (!LQ_IN_RANGE((size_t)(r * a + i) * L.ldz + j + 1,
+                                                       (size_t)R * a * L.ldz))
+                                        return;
                                       *z = make_float2(__double2float_rn(v0),
                                                        __double2float_rn(v1));
                                     });
@@ -523,7 +530,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
             store_codes<true>(q, s, m0 * row_chunks + ch, codes8, opf, codes4, scales,
                               K / kGroup, gs, asum);
         } else if (valid) {
-          store_codes<false>(q, s, m0 * row_chunks + ch, codes8, opf, codes4, scales);
+          if (LQ_IN_RANGE(m0 * row_chunks + ch, M * row_chunks))
+            store_codes<false>(q, s, m0 * row_chunks + ch, codes8, opf, codes4, scales);
         }
       }
     }
@@ -665,6 +673,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
                                       [&](int ri, int j, double v0, double v1) {
                                         const int r = (int)fd_a.div((uint32_t)ri), i = ri - r * a;
                                         double* yt = YT + ((size_t)r * b + j) * L.lda + i;
+                                        if (!LQ_IN_RANGE(((size_t)r * b + j + 1) * L.lda + i,
+                                                         (size_t)R * b * L.lda))
+                                          return;
                                         yt[0] = v0;
                                         yt[L.lda] = v1;
                                       });
@@ -680,6 +691,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
                                       [&](int i, int j, double v0, double v1) {
                                         float2* z = reinterpret_cast<float2*>(
                                             XZ + (size_t)(r * a + i) * L.ldz + j);
+                                        if (!LQ_IN_RANGE((size_t)(r * a + i) * L.ldz + j + 1,
+                                                         L.xz_floats))
+                                          return;
                                         *z = make_float2(__double2float_rn(v0),
                                                          __double2float_rn(v1));
                                       });
@@ -719,7 +733,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
         if (ch < n_chunks) {
           const int r = (int)fd_rowc.div((uint32_t)ch), k8 = (ch - r * row_chunks) * 8;
           const int i = (int)fd_b.div((uint32_t)k8), q = k8 - i * b;
-          xr[u].store(X + (size_t)(r * a + i) * L.ldb + q);
+          const size_t off = (size_t)(r * a + i) * L.ldb + q;
+          if (LQ_IN_RANGE(off + 7, L.xz_floats)) xr[u].store(X + off);
         }
       }
       for (int ch = kWsLoadU * kWsQThreads + qt; ch < n_chunks; ch += kWsQThreads) {
@@ -732,7 +747,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
         } else {
           v.zero();
         }
-        v.store(X + (size_t)(r * a + i) * L.ldb + q);
+        const size_t off = (size_t)(r * a + i) * L.ldb + q;
+        if (LQ_IN_RANGE(off + 7, L.xz_floats)) v.store(X + off);
       }
       if (qt < R) {
         const int64_t gr = m0 + qt, j = gr / segs.seg_rows;
@@ -765,7 +781,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
           if (valid) {
             const int k8 = (ch - r * row_chunks) * 8;
             const int i = (int)fd_b.div((uint32_t)k8), j = k8 - i * b;
-            const float4* src = reinterpret_cast<const float4*>(Z + (size_t)(r * a + i) * L.ldz + j);
+            const float4* src =
+                reinterpret_cast<const float4*>(Z + (size_t)(r * a + i) * L.ldz + j);
             const float4 u0 = src[0], u1 = src[1];
             v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
             v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
@@ -775,7 +792,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
           }
           uint32_t q[8];
           const float sc = quant_group8(v, c, qmax, q);
-          if (valid) store_codes<false>(q, sc, m0 * row_chunks + ch, codes8, opf, codes4, scales);
+          if (valid && LQ_IN_RANGE(m0 * row_chunks + ch, M * row_chunks))
+            store_codes<false>(q, sc, m0 * row_chunks + ch, codes8, opf, codes4, scales);
         }
         named_sync(kBarWsQ, kWsQThreads);  // Z(it - 2) and its clips fully read
       }
@@ -948,37 +966,54 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
   }
 }
 
-__global__ void k_codes4_to_operand(const uint8_t* __restrict__ codes4, int64_t n_words, int opf,
-                                    uint8_t* __restrict__ out) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_words; i += stride) {
-    const uint32_t w = reinterpret_cast<const uint32_t*>(codes4)[i];
-    uint32_t o0 = 0, o1 = 0;
+
+// The tensor-core GEMM's weight operand, expanded from the resident packed
+// codes for one launch: blocks [0, n_conv) turn packed words (8 codes) into
+// 8 code bytes (E4M3 or int8, as the GEMM's kind reads them); blocks from
+// n_conv on transpose the N x G steps into G x N in 32 x 32 tiles.  Under
+// programmatic dependent launch it waits for its predecessor before writing
+// (the previous GEMM of the sequence may still read the same workspace).
+__global__ void __launch_bounds__(256) k_weight_operand(
+    const uint8_t* __restrict__ codes4, int64_t n_words, int opf, uint8_t* __restrict__ op,
+    const float* __restrict__ sw, int64_t N, int64_t G, float* __restrict__ sw_t, int n_conv) {
+  pdl_trigger();
+  if ((int)blockIdx.x < n_conv) {
+    const int64_t stride = (int64_t)n_conv * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint32_t w = i0 < n_words ? __ldg(reinterpret_cast<const uint32_t*>(codes4) + i0) : 0u;
+    pdl_wait();
+    for (int64_t i = i0; i < n_words; i += stride) {
+      if (i != i0) w = __ldg(reinterpret_cast<const uint32_t*>(codes4) + i);
+      uint32_t o0 = 0, o1 = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      int nib = (int)((w >> (4 * j)) & 0xFu);
-      nib = nib >= 8 ? nib - 16 : nib;
-      const uint32_t byte = encode_code_byte(nib, opf);
-      if (j < 4) o0 |= byte << (8 * j); else o1 |= byte << (8 * (j - 4));
+      for (int j = 0; j < 8; ++j) {
+        int nib = (int)((w >> (4 * j)) & 0xFu);
+        nib = nib >= 8 ? nib - 16 : nib;
+        const uint32_t byte = encode_code_byte(nib, opf);
+        if (j < 4) o0 |= byte << (8 * j); else o1 |= byte << (8 * (j - 4));
+      }
+      reinterpret_cast<uint2*>(op)[i] = make_uint2(o0, o1);
     }
-    reinterpret_cast<uint2*>(out)[i] = make_uint2(o0, o1);
+    return;
+  }
+  // steps: tile t of the (N / 32 rounded up) x (G / 32 rounded up) tiles
+  __shared__ float tile[32][33];
+  const int64_t t = (int64_t)blockIdx.x - n_conv;
+  const int64_t tiles_g = (G + 31) / 32;
+  const int64_t r0 = (t / tiles_g) * 32, c0 = (t % tiles_g) * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t r = r0 + i, cc = c0 + tx;
+    if (r < N && cc < G) tile[i][tx] = __ldg(sw + r * G + cc);
+  }
+  __syncthreads();
+  pdl_wait();
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t cc = c0 + i, r = r0 + tx;
+    if (r < N && cc < G) sw_t[cc * N + r] = tile[tx][i];
   }
 }
 
-__global__ void k_transpose_f32(const float* __restrict__ in, int64_t rows, int64_t cols,
-                                float* __restrict__ out) {
-  __shared__ float tile[32][33];
-  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int64_t r = r0 + i, cc = c0 + threadIdx.x;
-    if (r < rows && cc < cols) tile[i][threadIdx.x] = in[r * cols + cc];
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int64_t cc = c0 + i, r = r0 + threadIdx.x;
-    if (r < rows && cc < cols) out[cc * rows + r] = tile[threadIdx.x][i];
-  }
-}
 
 template <typename F>
 cudaError_t set_smem(F* f, size_t bytes) {
@@ -1133,21 +1168,19 @@ cudaError_t launch_rotate_store(const float* x, int64_t M, int64_t K, const floa
   return cudaGetLastError();
 }
 
-cudaError_t launch_codes4_to_operand(const uint8_t* codes4, int64_t n_bytes, int opf,
-                                     uint8_t* out, cudaStream_t s) {
-  const int64_t n_words = n_bytes / 4;
+
+cudaError_t launch_weight_operand(const uint8_t* codes4, const float* sw, int64_t N, int64_t K,
+                                  int opf, uint8_t* op, float* sw_t, cudaStream_t s, bool pdl) {
+  const int64_t n_words = N * K / 8, G = K / kGroup;
   if (n_words == 0) return cudaSuccess;
-  const int grid = (int)std::min<int64_t>((n_words + 255) / 256, (int64_t)num_sms() * 16);
-  k_codes4_to_operand<<<grid, 256, 0, s>>>(codes4, n_words, opf, out);
-  return cudaGetLastError();
+  const int n_conv = (int)std::min<int64_t>((n_words + 255) / 256, (int64_t)num_sms() * 8);
+  const int64_t n_tr = ((N + 31) / 32) * ((G + 31) / 32);
+  if (n_conv + n_tr > INT32_MAX) return cudaErrorInvalidValue;
+  return launch_kernel(k_weight_operand, dim3((unsigned)(n_conv + n_tr)), dim3(256), 0, s, pdl,
+                       codes4, n_words, opf, op, sw, N, G, sw_t, n_conv);
 }
 
-cudaError_t launch_transpose_f32(const float* in, int64_t rows, int64_t cols, float* out,
-                                 cudaStream_t s) {
-  if (rows == 0 || cols == 0) return cudaSuccess;
-  dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows + 31) / 32));
-  k_transpose_f32<<<grid, dim3(32, 8), 0, s>>>(in, rows, cols, out);
-  return cudaGetLastError();
-}
+
+unsigned long long bounds_fail_quant() { return lq_take_bounds_fail(); }
 
 }  // namespace lq

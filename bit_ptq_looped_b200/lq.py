@@ -22,12 +22,13 @@ LIB_PATH = os.environ.get("LQ_LIB_PATH") or os.path.join(HERE, "liblq.so")
 
 LQ_OK, LQ_ERR_ARG, LQ_ERR_SHAPE, LQ_ERR_UNSUPPORTED, LQ_ERR_ALIGN = 0, 1, 2, 3, 4
 LQ_ERR_CUDA, LQ_ERR_DEVICE_TIMEOUT, LQ_ERR_NOMEM, LQ_ERR_WORKSPACE = 5, 6, 7, 8
+LQ_ERR_DEVICE_BOUNDS = 9
 LQ_F32, LQ_BF16 = 0, 1
 LQ_OPEN, LQ_CHAIN = 0, 1
 
 STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_ARG", 2: "LQ_ERR_SHAPE", 3: "LQ_ERR_UNSUPPORTED",
                 4: "LQ_ERR_ALIGN", 5: "LQ_ERR_CUDA", 6: "LQ_ERR_DEVICE_TIMEOUT",
-                7: "LQ_ERR_NOMEM", 8: "LQ_ERR_WORKSPACE"}
+                7: "LQ_ERR_NOMEM", 8: "LQ_ERR_WORKSPACE", 9: "LQ_ERR_DEVICE_BOUNDS"}
 
 # symbol -> (restype, argtypes)
 _vp, _i32, _i64, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
@@ -66,7 +67,7 @@ SIGNATURES = {
     "lq_probe_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]),
 }
 
-PROBE_KINDS = ("rotate_quantize", "quantize", "gemm", "gemv")
+PROBE_KINDS = ("rotate_quantize", "quantize", "gemm", "gemv", "weight_operand")
 
 _lib: Optional[ctypes.CDLL] = None
 

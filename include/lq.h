@@ -56,6 +56,7 @@ typedef int32_t lq_status;
 #define LQ_ERR_DEVICE_TIMEOUT  6  /* a bounded device-side wait expired         */
 #define LQ_ERR_NOMEM           7  /* device allocation failed                   */
 #define LQ_ERR_WORKSPACE       8  /* workspace too small                        */
+#define LQ_ERR_DEVICE_BOUNDS   9  /* bounds-check build: a kernel index out of range */
 
 /* element types of activation inputs */
 #define LQ_F32   0
@@ -136,8 +137,10 @@ lq_status lq_quantize_weights(const float* d_W, int64_t N, int64_t K, int32_t bi
  * lq_pack_weights -- quantize folded weights into a library-owned resident
  * object used by every loop.  Allocates device memory (cudaMalloc); the call
  * synchronises `stream` before returning.  Release with lq_wq_free.
- * Resident layout: packed 4-bit codes N x K/2, scales N x G and G x N
- * (float32), and the tensor-core operand copy created by lq_layer_create.
+ * Resident layout: packed 4-bit codes N x K/2 and their steps N x G
+ * (float32): 0.625 bytes per weight.  Calls that run the tensor-core GEMM
+ * expand, per launch, an 8-bit operand copy (N x K bytes) and the steps
+ * transposed (G x N) into their workspace; nothing else is kept resident.
  */
 lq_status lq_pack_weights(const float* d_W_folded, int64_t N, int64_t K, int32_t bits,
                           int32_t group, lq_wq** out, void* stream);
@@ -154,8 +157,8 @@ void lq_wq_free(lq_wq* wq);
 /*
  * lq_layer_create -- bind resident weights to a module's Kronecker factors
  * and LAS clips.  Copies P1 (a x a), P2 (b x b) (device pointers) and
- * h_las[T] (host, every entry > 0) into library-owned device memory and
- * prepares the tensor-core operand copy of the weights for a_bits (4 or 8).
+ * h_las[T] (host, every entry > 0) into library-owned device memory;
+ * a_bits (4 or 8) selects the activation precision.
  * Synchronous.  `wq` must outlive the layer.  a*b must equal wq's K.
  */
 lq_status lq_layer_create(const lq_wq* wq, const float* d_P1, int32_t a, const float* d_P2,
@@ -165,15 +168,21 @@ void lq_layer_free(lq_layer* layer);
 
 /*
  * Device workspace needed by lq_loop_linear / lq_loop_stack for M tokens
- * through the given layers (the activation codes and steps of one step).
+ * through the given layers: the activation codes and steps of one step, and
+ * for the tensor-core path (M > 16) the weight operand of the largest layer
+ * (N x K code bytes + G x N steps), expanded from the resident 4-bit codes by
+ * each call.
  */
 int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M);
 
 /*
  * Workspace with which lq_loop_stack in LQ_OPEN mode runs up to min(T, 8)
  * loops of each layer in one quantize and one GEMM launch (the loops of a
- * layer are independent in open mode and share the resident weights).  Equal
- * to lq_workspace_bytes for decode-sized M (the GEMV path runs loop by loop).
+ * layer are independent in open mode and share the resident weights).  For
+ * decode-sized M (the GEMV path, M <= 16) it is the size that lets the
+ * independent (t, l) steps of open mode run as up to 16 concurrent
+ * quantize->GEMV chains, each with its own slice (smaller workspaces run
+ * fewer chains, one at least).
  * Returns -1 on a null pointer or a non-positive L or T.
  */
 int64_t lq_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M,
@@ -200,8 +209,10 @@ lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_l
  *   d_ws  at least lq_workspace_bytes(layers, L, M) bytes, 256-byte aligned.
  *         In LQ_OPEN mode a larger workspace lets one launch cover several
  *         loops of a layer (as many as fit, at most 8;
- *         lq_stack_workspace_bytes gives the size for min(T, 8)); results are
- *         the same either way.
+ *         lq_stack_workspace_bytes gives the size for min(T, 8)), or, for
+ *         decode-sized M, lets up to 16 (t, l) steps run concurrently on
+ *         internal streams forked from and joined back into `stream`;
+ *         results are the same either way.
  * Consecutive kernels of the schedule use programmatic dependent launch: a
  * kernel starts its prologue (weight loads, rotation of inputs that exist
  * before the call) while its predecessor finishes, and waits for it before
@@ -318,7 +329,8 @@ lq_status lq_trajectory_hessian(const void* d_X, int32_t x_dtype, int64_t M, int
  * built into the library; every GPU that loads the library holds it until the
  * process exits.  The call allocates nothing (no cudaMalloc, no cudaFree).
  *   - Calls needing more scratch than that, lq_workspace_bytes(&layer, 1, M)
- *     > LQ_NOALLOC_SCRATCH_BYTES (about M*K*(1 + 1/8) bytes), fail with
+ *     > LQ_NOALLOC_SCRATCH_BYTES (about M*K*(1 + 1/8) bytes, plus
+ *     N*K*(1 + 1/8) for the weight operand when M > 16), fail with
  *     LQ_ERR_WORKSPACE and enqueue nothing.
  *   - All calls share the one array, which keeps the last call's contents.
  *     Each call writes every scratch byte it reads before reading it, so
@@ -340,17 +352,23 @@ lq_status lq_loop_linear_noalloc(const void* d_x, int32_t x_dtype, int64_t M,
  * with CUDA events recorded on the launching stream.  lq_probe_read waits for
  * those events and returns, per kernel kind, the summed device time in
  * milliseconds and the number of launches, then clears them.  Kinds (index):
- * 0 fused rotate+quantize, 1 quantize-only, 2 tensor-core GEMM, 3 GEMV.
+ * 0 fused rotate+quantize, 1 quantize-only, 2 tensor-core GEMM, 3 GEMV,
+ * 4 weight-operand expansion (the GEMM's 8-bit weight bytes and transposed
+ * steps, one per GEMM launch).
  * h_ms and h_count point to arrays of LQ_PROBE_KINDS entries (host memory).
  */
-#define LQ_PROBE_KINDS 4
+#define LQ_PROBE_KINDS 5
 lq_status lq_probe_enable(int32_t on);
 lq_status lq_probe_read(double* h_ms, int64_t* h_count);
 
 /*
  * lq_check_device -- synchronise `stream`, then read and clear the device
  * status word that kernels set when a bounded wait expires.  Returns LQ_OK or
- * LQ_ERR_DEVICE_TIMEOUT (or LQ_ERR_CUDA for an asynchronous CUDA error).
+ * LQ_ERR_DEVICE_TIMEOUT (or LQ_ERR_CUDA for an asynchronous CUDA error).  In
+ * the bounds-check build (compiled with -DLQ_BOUNDS_CHECK) kernels also test
+ * their store indices against the extents they write, skip and record an
+ * index out of range, and this call returns LQ_ERR_DEVICE_BOUNDS with the
+ * source line and index in lq_last_error(); the normal build never does.
  */
 lq_status lq_check_device(void* stream);
 

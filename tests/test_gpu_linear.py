@@ -159,6 +159,21 @@ def test_loop_linear_ragged_rows(M):
     linear_parity(host(y), x, ol, 2, host(q8), host(s), layer.w_flips)
 
 
+def test_resident_weights_are_four_bit():
+    """The resident weight object holds only the packed 4-bit codes and their
+    float32 steps: N*K/2 + N*(K/32)*4 bytes, 0.625 bytes per weight; the
+    tensor-core path expands its 8-bit operand into the call's workspace."""
+    wl = synth.MLP
+    for mp in synth.module_params(wl):
+        layer, _ = make_layer(mp, 4)
+        info = layer.wq.info()
+        N, K = info["N"], info["K"]
+        assert info["device_bytes"] == N * K // 2 + N * (K // 32) * 4
+        assert info["device_bytes"] / (N * K) <= 0.66
+        M = 256  # tensor-core path: the workspace holds the operand of this layer
+        assert lq.lq_workspace_bytes([layer], M) >= M * K + N * K
+
+
 def test_loop_linear_rejects_bad_calls():
     wl = synth.TINY
     (mp,) = synth.module_params(wl)
@@ -232,10 +247,50 @@ def test_loop_stack_open_batching_matches_per_loop(wl, M):
     ref = lq.lq_loop_stack(xd, layers, T, lq.LQ_OPEN, M=M, ws=lq.workspace(layers, M))
     for nb in (2, 3, T):
         ws = lq.workspace(layers, M, T=nb)
-        assert ws.numel() >= lq.lq_workspace_bytes(layers, M) * (nb - 0.5)
+        # room for the codes and steps of nb loops (beside one weight operand)
+        kmax = max(lin.K for lin in wl.linears)
+        assert ws.numel() >= lq.lq_workspace_bytes(layers, M) + (nb - 1) * M * kmax
         y = lq.lq_loop_stack(xd, layers, T, lq.LQ_OPEN, M=M, ws=ws)
         torch.cuda.synchronize()
         assert torch.equal(y, ref), f"batch of {nb} loops"
+
+
+@pytest.mark.parametrize("M,a_bits", [(1, 8), (4, 4), (16, 8)])
+def test_loop_stack_open_decode_branches(M, a_bits):
+    """Decode-sized open mode: the T x L independent (t, l) steps run as
+    concurrent quantize->GEMV chains on internal streams, each with its own
+    workspace slice.  Three linears of different widths (the last with a
+    ragged N), T = 4: every output against the oracle, and bit-identical to
+    the one-chain schedule a minimal workspace gives (same kernels per step)."""
+    lins = (synth.Linear("d0", 2048, 2048, 32, 64, 0), synth.Linear("d1", 2048, 5632, 32, 64, 0),
+            synth.Linear("d2", 2048, 1000, 32, 64, 1))
+    wl = synth.Workload(f"decode_stack_M{M}", M=M, T=4, linears=lins, a_bits=a_bits,
+                        outlier_frac=0.02, outlier_mult=20.0, x_dtype="bf16",
+                        description="decode stack of three linears")
+    params = synth.module_params(wl)
+    built = [make_layer(mp, a_bits) for mp in params]
+    layers = [b[0] for b in built]
+    xs, flat = _stack_inputs(wl, M)
+    xd = act_tensor(flat, wl.x_dtype)
+    ws_all = lq.workspace(layers, M, T=wl.T)
+    ws_one = lq.workspace(layers, M)
+    assert ws_all.numel() >= 12 * ws_one.numel() // 2
+    y = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, ws=ws_all)
+    y1 = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, ws=ws_one)
+    y2 = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, ws=ws_all, y=torch.empty_like(y))
+    torch.cuda.synchronize()
+    assert torch.equal(y, y1) and torch.equal(y, y2)
+    yh = host(y)
+    off = 0
+    for t in range(wl.T):
+        for l, (lin, mp) in enumerate(zip(wl.linears, params)):
+            n = M * lin.N
+            yg = yh[off:off + n].reshape(M, lin.N)
+            off += n
+            q8, _, s = lq.lq_quantize_act(act_tensor(xs[t][l], wl.x_dtype), dev(mp.P1),
+                                          dev(mp.P2), float(mp.las[t]), a_bits)
+            torch.cuda.synchronize()
+            linear_parity(yg, xs[t][l], built[l][1], t, host(q8), host(s), built[l][0].w_flips)
 
 
 def test_loop_stack_open_more_than_eight_loops():
