@@ -732,6 +732,32 @@ def aux_schedules(lq, ctx, wl, layers, x_dev, ops_step):
     return out
 
 
+def aux_decode_chain(lq, ctx, peaks, M=4, L=32):
+    """Decode as a real looped model runs it: chain mode, each (t, l) step's
+    input the previous step's output, so the T x L quantize -> GEMV pairs are
+    strictly sequential (K = N = 2048, L distinct resident copies, W4A8)."""
+    torch = ctx.torch
+    wl = synth.decode_workload(M, 2048, 8)
+    layers, packed = build_layers(lq, torch, ctx.dev, wl, L)
+    x0 = torch.from_numpy(synth.loop_input(wl, wl.linears[0], 0)).to(torch.bfloat16).to(ctx.dev)
+    y = torch.empty(wl.T * L * M * 2048, dtype=torch.float32, device=ctx.dev)
+    ws = lq.workspace(layers, M, ctx.dev)
+
+    def step():
+        lq.lq_loop_stack(x0, layers, wl.T, lq.LQ_CHAIN, M=M, y=y, ws=ws, stream=ctx.stream)
+
+    for _ in range(3):
+        step()
+    n = 20
+    ms = ctx.timed(n, step) / n
+    free_layers(layers, packed)
+    wb = 2048 * 2048 * 5 // 8
+    return {"workload": f"W4A8 M={M} K=N=2048, chain mode, T={wl.T} x {L} distinct linears",
+            "ms_per_step": ms, "us_per_linear": ms * 1e3 / (wl.T * L),
+            "tokens_per_s": M / (ms * 1e-3),
+            "weight_stream_frac_hbm": wl.T * L * wb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+
+
 def aux_hbm_kernels(lq, ctx, peaks):
     """The quantize-only kernel and the streaming GEMV on launches far larger than L2."""
     torch, dev, stream = ctx.torch, ctx.dev, ctx.stream
@@ -846,6 +872,7 @@ def run_lq(args, rank, world, local_rank):
             del a_held
             aux[name] = a_line
         torch.cuda.empty_cache()
+        aux["decode_chain_M4_N2048"] = aux_decode_chain(lq, ctx, peaks)
         aux.update(aux_hbm_kernels(lq, ctx, peaks))
 
     cpu = None

@@ -562,11 +562,15 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
 // Shared memory: P2T [b][b+4] and P1T [a][a+4] (float64), YT [R][b][a+4]
 // (float64, MMA warps only), and two X/Z buffers of R*a rows x (b+4) floats.
 // ---------------------------------------------------------------------------
-constexpr int kWsMmaWarps = 8;
+// Two configurations (template arguments), chosen per factor shape at launch:
+// 8 MMA warps with 16 x 32 warp tasks (more independent MMA chains per warp)
+// when both stages split evenly over 8 warps, else 12 MMA warps with 16 x 16
+// tasks (32 x 64 factors: 4 % faster with the wide tasks; 64 x 88: 4 % with
+// 12 warps).
 constexpr int kWsQWarps = 4;
-constexpr int kWsMmaThreads = 32 * kWsMmaWarps;
 constexpr int kWsQThreads = 32 * kWsQWarps;
-constexpr int kWsThreads = kWsMmaThreads + kWsQThreads;
+template <int kMmaWarps>
+__host__ __device__ constexpr int ws_threads() { return 32 * (kMmaWarps + kWsQWarps); }
 constexpr int kWsLoadU = 8;  // input chunks (8 elements) per quant thread in flight
 constexpr size_t kWsSmemLimit = 226u * 1024u;  // dynamic shared memory of one block
 // named barrier ids (0 is __syncthreads)
@@ -603,12 +607,14 @@ __host__ __device__ inline WsLayout ws_layout(int a, int b, int R) {
   return L;
 }
 
-template <typename Tin>
-__global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
+template <typename Tin, int kTN, int kWsMmaWarps>
+__global__ void __launch_bounds__(ws_threads<kWsMmaWarps>(), 1) k_rotate_quant_ws(
     const Tin* __restrict__ x, int64_t M, int K, const float* __restrict__ P1, int a,
     const float* __restrict__ P2, int b, int R, const LoopSegs segs, int qmax,
     int8_t* __restrict__ codes8, int opf, uint8_t* __restrict__ codes4,
     float* __restrict__ scales, int x_early) {
+  constexpr int kWsMmaThreads = 32 * kWsMmaWarps;
+  constexpr int kWsThreads = ws_threads<kWsMmaWarps>();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   pdl_trigger();
   if (!x_early) pdl_wait();
@@ -657,7 +663,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
   if (warp < kWsMmaWarps) {
     // ---------------- MMA warps ----------------
     const int ct = b >> 3;
-    const int s1_ctq = (ct + kRotTN - 1) / kRotTN;
+    const int s1_ctq = (ct + kTN - 1) / kTN;
     const int s1_tasks = ((R * a) / (8 * kRotTM)) * s1_ctq;
     const int s2_rt = a / (8 * kRotTM);
     const int s2_tasks = R * s2_rt * s1_ctq;
@@ -669,7 +675,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
       // stage 1: Y[(r,i), j] = sum_q X[(r,i), q] P2[q, j]  -> YT[r][j][i]
       for (int task = warp; task < s1_tasks; task += kWsMmaWarps) {
         const int rt = (int)fd_s1ctq.div((uint32_t)task), cq = task - rt * s1_ctq;
-        warp_mma_task<kRotTM, kRotTN>(XZ, L.ldb, P2T, L.ldb, b, rt * 8 * kRotTM, cq * kRotTN, ct,
+        warp_mma_task<kRotTM, kTN>(XZ, L.ldb, P2T, L.ldb, b, rt * 8 * kRotTM, cq * kTN, ct,
                                       [&](int ri, int j, double v0, double v1) {
                                         const int r = (int)fd_a.div((uint32_t)ri), i = ri - r * a;
                                         double* yt = YT + ((size_t)r * b + j) * L.lda + i;
@@ -686,8 +692,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_rotate_quant_ws(
         const int r = (int)fd_s2tok.div((uint32_t)task);
         const int rem = task - r * (s2_rt * s1_ctq);
         const int rt = (int)fd_s1ctq.div((uint32_t)rem), cq = rem - rt * s1_ctq;
-        warp_mma_task<kRotTM, kRotTN>(P1T, L.lda, YT + (size_t)r * b * L.lda, L.lda, a,
-                                      rt * 8 * kRotTM, cq * kRotTN, ct,
+        warp_mma_task<kRotTM, kTN>(P1T, L.lda, YT + (size_t)r * b * L.lda, L.lda, a,
+                                      rt * 8 * kRotTM, cq * kTN, ct,
                                       [&](int i, int j, double v0, double v1) {
                                         float2* z = reinterpret_cast<float2*>(
                                             XZ + (size_t)(r * a + i) * L.ldz + j);
@@ -1109,18 +1115,24 @@ cudaError_t launch_quantize(const void* x, int x_dtype, int64_t M, int64_t K, co
       const size_t wsm = ws_layout(a, b, Rw).bytes;
       const int64_t tiles = (M + Rw - 1) / Rw;
       const int grid = (int)std::min<int64_t>(tiles, (int64_t)num_sms());
-      cudaError_t e;
+      // wide warp tasks on 8 MMA warps when both stages split evenly, else 12 warps
+      const int ctq4 = ((b >> 3) + 3) / 4;
+      const bool wide = (b >> 3) % 4 == 0 && ((Rw * a) / 16 * ctq4) % 8 == 0 &&
+                        (Rw * (a / 16) * ctq4) % 8 == 0;
+      auto go = [&](auto* k, int threads, const auto* xin) -> cudaError_t {
+        cudaError_t e = set_smem(k, wsm);
+        if (e != cudaSuccess) return e;
+        return launch_kernel(k, dim3(grid), dim3(threads), wsm, s, pdl, xin, M, (int)K, P1, a,
+                             P2, b, Rw, segs, qmax, codes8, opf, codes4, scales, xe);
+      };
       if (x_dtype == LQ_BF16) {
-        auto* k = k_rotate_quant_ws<__nv_bfloat16>;
-        if ((e = set_smem(k, wsm)) != cudaSuccess) return e;
-        return launch_kernel(k, dim3(grid), dim3(kWsThreads), wsm, s, pdl,
-                             (const __nv_bfloat16*)x, M, (int)K, P1, a, P2, b, Rw, segs, qmax,
-                             codes8, opf, codes4, scales, xe);
+        const auto* xb = (const __nv_bfloat16*)x;
+        return wide ? go(k_rotate_quant_ws<__nv_bfloat16, 4, 8>, ws_threads<8>(), xb)
+                    : go(k_rotate_quant_ws<__nv_bfloat16, 2, 12>, ws_threads<12>(), xb);
       }
-      auto* k = k_rotate_quant_ws<float>;
-      if ((e = set_smem(k, wsm)) != cudaSuccess) return e;
-      return launch_kernel(k, dim3(grid), dim3(kWsThreads), wsm, s, pdl, (const float*)x, M,
-                           (int)K, P1, a, P2, b, Rw, segs, qmax, codes8, opf, codes4, scales, xe);
+      const auto* xf = (const float*)x;
+      return wide ? go(k_rotate_quant_ws<float, 4, 8>, ws_threads<8>(), xf)
+                  : go(k_rotate_quant_ws<float, 2, 12>, ws_threads<12>(), xf);
     }
   }
   int R = 0;
