@@ -97,6 +97,34 @@ def test_loop_stack_cta_tiny_matches_oracle():
     cta.free()
 
 
+@pytest.mark.parametrize("M", [300, 2048])
+def test_loop_stack_cta_two_pass_state_matches_oracle(M):
+    """The adapted state the last transition of the chained schedule leaves in
+    the workspace (right after the codes and steps) must equal the oracle's
+    CTA of that loop's output (both round a float64 value once: at most one
+    unit in the last place on at most 1e-4 of the values); d = 2048, a ragged
+    last 8-row block at M = 300."""
+    from tests.test_gpu_linear import make_layer
+    wl = synth.ATTN_PROJ
+    (mp,) = synth.module_params(wl)
+    layer, _ = make_layer(mp, 4)
+    d, T = 2048, 3
+    U, V, a, b, eta = _adapter(d, 8, T - 1, seed=M)
+    cta = lq.lq_cta_create(dev(U), dev(V), dev(a), dev(b), eta)
+    x0 = dev(synth.loop_input(wl, wl.linears[0], 0, rows=np.arange(M)))
+    nws = lq.lq_cta_stack_workspace_bytes([layer], M)
+    ws = torch.zeros(nws, dtype=torch.uint8, device="cuda")
+    y = host(lq.lq_loop_stack_cta(x0, [layer], T, cta, M=M, ws=ws))
+    torch.cuda.synchronize()
+    off = -(-lq.lq_workspace_bytes([layer], M) // 256) * 256
+    state = host(ws[off:off + M * d * 4].view(torch.float32)).reshape(M, d)
+    y_last = y[(T - 2) * M * d:(T - 1) * M * d].reshape(M, d)
+    ref = O.cta_apply(y_last, a[T - 2], b[T - 2], float(eta[T - 2]), U, V)
+    du = _ulp_diff(state, ref)
+    assert du.max() <= 1 and (du > 0).mean() <= 1e-4, (du.max(), (du > 0).mean())
+    cta.free()
+
+
 def test_loop_stack_cta_identity_is_plain_chain():
     wl, mp, (layer, ol) = _tiny_layer()
     (lin,) = wl.linears
