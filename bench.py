@@ -457,10 +457,15 @@ def roofline_of(kernels, wl, n_probe, copies, peaks, sustained):
         peak = SM_COUNT * FP64_FMA_PER_SM_CLK * 2 * SM_CLOCK_GHZ * 1e9 / 1e12
         r = {"bound": "alu", "achieved": flops / avg_s / 1e12, "peak": peak,
              "unit": "TFLOP/s", "peak_source": "derived: 148 SM x 64 FP64 FMA/clk x 2 x 1.965 GHz"}
-    else:  # GEMV: the weight stream (packed codes + steps) per launch, no L2 credit
-        byts = sum(lin.N * lin.K * 5 // 8 * T for lin in wl.linears) * copies / per_step
+    else:  # GEMV: one linear's weight stream (packed codes + steps) per launch, whatever
+        # the number of loops batched into it, plus its float32 outputs; no L2 credit
+        n_lin = len(wl.linears)
+        wbytes = sum(lin.N * lin.K * 5 // 8 for lin in wl.linears) / n_lin
+        ybytes = rows_per_launch / n_lin * sum(lin.N * 4 for lin in wl.linears) / n_lin
+        byts = wbytes + ybytes
         r = {"bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
-             "unit": "GB/s", "peak_source": peaks["source"] + " copy bandwidth"}
+             "unit": "GB/s", "peak_source": peaks["source"] + " copy bandwidth",
+             "bytes_per_launch": byts}
     r["frac"] = r["achieved"] / r["peak"]
     r["kernel"] = dom
     r["traffic"] = ncu_traffic(dom, wl.name, rows_per_launch)
@@ -609,13 +614,20 @@ def measure_stack(lq, ctx, wl, n_steps, warmup, n_probe, peaks, want_clocks=Fals
             "tokens_per_s": wl.M * copies * ctx.world / (ms * 1e-3),
             "rotation_tflops": rot * ctx.world / (ms * 1e-3) / 1e12,
             "clocks": clocks, "steps": n_steps, "config": workload_config(wl, ctx.world, copies)}
+    kernels = probe_kernels(lq, ctx, step, n_probe, not big) if n_probe else None
     if is_decode(wl):
         xb, wb, yb = step_bytes(wl, copies)
-        line["weight_stream_GB_s"] = wl.T * wb / (ms * 1e-3) / 1e9
+        # weight passes per step: one per GEMV launch of a linear (the loops
+        # batched into a launch share its pass), counted by the probe
+        passes = wl.T
+        if kernels and "gemv" in kernels:
+            passes = kernels["gemv"]["launches"] / n_probe / (copies * len(wl.linears))
+        line["weight_passes_per_step"] = passes
+        line["weight_bytes_per_step"] = passes * wb
+        line["weight_stream_GB_s"] = passes * wb / (ms * 1e-3) / 1e9
         line["weight_stream_frac_hbm"] = line["weight_stream_GB_s"] / peaks["hbm_gbs"]
         line["tokens_per_s_per_linear"] = wl.M / (ms * 1e-3 / copies)
-    if n_probe:
-        kernels = probe_kernels(lq, ctx, step, n_probe, not big)
+    if kernels:
         line["kernels"] = kernels
         line["launches_per_step"] = sum(v["launches"] for v in kernels.values()) / n_probe
         line["roofline"] = roofline_of(kernels, wl, n_probe, copies, peaks,

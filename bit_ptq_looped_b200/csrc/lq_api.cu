@@ -282,8 +282,8 @@ lq_status enqueue_linear(const void* x, int32_t x_dtype, int64_t M, const lq_lay
   uint8_t* codes = (uint8_t*)ws;
   float* scales = (float*)((char*)ws + round_up(Mt * K, 256));
   int* asum = gemv ? (int*)((char*)scales + round_up(Mt * (K / kGroup) * 4, 256)) : nullptr;
-  if (nb > 1 && (gemv || L->P1 == nullptr || nb > kMaxLoopsPerLaunch)) {
-    set_error("internal: loop batching needs the rotating tensor-core path");
+  if (nb > 1 && (L->P1 == nullptr || nb > kMaxLoopsPerLaunch)) {
+    set_error("internal: loop batching needs the rotating quantizer");
     return LQ_ERR_ARG;
   }
   LoopSegs segs = one_loop(L->las[t]);
@@ -303,8 +303,8 @@ lq_status enqueue_linear(const void* x, int32_t x_dtype, int64_t M, const lq_lay
   if (e != cudaSuccess) return cuda_error(e, "quantize launch");
   if (gemv) {
     ProbeScope ps(kProbeGemv, s);
-    e = launch_group_gemv((const int8_t*)codes, asum, scales, wq->codes4, wq->scales, y, M, N, K,
-                          s, pdl);
+    e = launch_group_gemv((const int8_t*)codes, asum, scales, wq->codes4, wq->scales, y, Mt, N, K,
+                          s, pdl, nb > 1 ? M : INT64_MAX, y_stride);
     if (e != cudaSuccess) return cuda_error(e, "gemv launch");
   } else {
     // the weight operand for this launch, expanded from the resident 4-bit codes
@@ -331,14 +331,31 @@ lq_status enqueue_linear(const void* x, int32_t x_dtype, int64_t M, const lq_lay
 }
 
 // Loops of one layer that open mode runs per launch with a workspace of
-// ws_bytes: batching needs the rotating tensor-core path for M rows.
+// ws_bytes.  Batching needs the rotating quantizer (its per-loop row
+// segments); a decode-sized M stays on the GEMV path, so its batch is bounded
+// by the GEMV's row limit, and each launch then streams the layer's weights
+// once for all loops of the batch.
 int loops_per_launch(const lq_layer* L, int64_t M, int T, int64_t ws_bytes) {
   const int64_t K = L->wq->K;
-  if (use_gemv(M, K) || L->P1 == nullptr) return 1;
+  if (L->P1 == nullptr) return 1;
+  const bool gemv = use_gemv(M, K);
   int nb = std::min(T, kMaxLoopsPerLaunch);
-  while (nb > 1 && (ws_bytes_linear(M * nb, K, L->wq->N) > ws_bytes ||
+  while (nb > 1 && ((gemv && !use_gemv(M * nb, K)) ||
+                    ws_bytes_linear(M * nb, K, L->wq->N) > ws_bytes ||
                     M * nb > ((int64_t)1 << 31) - 256))
     --nb;
+  return nb;
+}
+
+// Loops per GEMV launch of a decode-sized open-mode stack: the most loops of
+// every layer whose rows still fit the GEMV path (1 when a layer does not
+// rotate).
+int decode_loops_per_launch(const std::vector<const lq_layer*>& tl, int64_t M, int T) {
+  int nb = std::min(T, kMaxLoopsPerLaunch);
+  for (const lq_layer* ly : tl) {
+    if (ly->P1 == nullptr) return 1;
+    while (nb > 1 && !use_gemv(M * nb, ly->wq->K)) --nb;
+  }
   return nb;
 }
 
@@ -687,16 +704,17 @@ int64_t lq_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64
   for (int i = 0; i < L; ++i) {
     if (!layers[i]) return -1;
     const int64_t K = layers[i]->wq->K;
-    const bool batch = !use_gemv(M, K) && layers[i]->P1 != nullptr;
-    const int nb = batch ? std::min<int>(T, kMaxLoopsPerLaunch) : 1;
+    const int nb = loops_per_launch(layers[i], M, T, INT64_MAX);
     need = std::max(need, ws_bytes_linear(M * nb, K, layers[i]->wq->N));
   }
   bool decode = (int64_t)T * L > 1;
   for (int i = 0; i < L; ++i) decode = decode && use_gemv(M, layers[i]->wq->K);
-  if (decode) {  // one workspace slice per concurrent decode chain
-    const std::vector<const lq_layer*> tl(layers, layers + L);
-    need = std::max(need, decode_branch_bytes(tl, M) *
-                              std::min<int64_t>(kDecodeBranches, (int64_t)T * L));
+  const std::vector<const lq_layer*> tl(layers, layers + L);
+  if (decode) {  // one workspace slice per concurrent decode chain of loop-batched steps
+    const int nbd = decode_loops_per_launch(tl, M, T);
+    const int64_t units = (int64_t)((T + nbd - 1) / nbd) * L;
+    need = std::max(need, decode_branch_bytes(tl, M * nbd) *
+                              std::min<int64_t>(kDecodeBranches, units));
   }
   return need;
 }
@@ -745,8 +763,28 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
     bool decode = T * L > 1;
     for (const lq_layer* ly : tl) decode = decode && use_gemv(M, ly->wq->K);
     if (decode) {
-      const int64_t per = decode_branch_bytes(tl, M);
-      const int nbr = (int)std::min(std::min((int64_t)kDecodeBranches, (int64_t)T * L),
+      // units of work: the loops t .. t + nbd - 1 of layer l in one quantize
+      // and one GEMV launch (the weights streamed once for them) when the
+      // same handle serves all of them, else one unit per loop
+      int nbd = decode_loops_per_launch(tl, M, T);
+      int64_t per = decode_branch_bytes(tl, M * nbd);
+      while (nbd > 1 && ws_bytes < 2 * per) per = decode_branch_bytes(tl, M * --nbd);
+      struct Unit {
+        int t, l, w;
+      };
+      std::vector<Unit> units;
+      for (int t = 0; t < T; t += nbd) {
+        const int nb = std::min(nbd, T - t);
+        for (int l = 0; l < L; ++l) {
+          bool same = true;
+          for (int j = 1; j < nb; ++j) same = same && at(t + j, l) == at(t, l);
+          if (same)
+            units.push_back({t, l, nb});
+          else
+            for (int j = 0; j < nb; ++j) units.push_back({t + j, l, 1});
+        }
+      }
+      const int nbr = (int)std::min(std::min((int64_t)kDecodeBranches, (int64_t)units.size()),
                                     ws_bytes / per);
       if (nbr >= 2) {
         std::lock_guard<std::mutex> lk(g_branch_mu);
@@ -758,20 +796,20 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
         for (int b = 0; b < nbr; ++b)
           if ((e = cudaStreamWaitEvent(bs->st[b], bs->fork, 0)) != cudaSuccess)
             return cuda_error(e, "fork wait");
-        int i = 0;
-        for (int t = 0; t < T && st == LQ_OK; ++t) {
-          int64_t k_before = 0, n_before = 0;
-          for (int l = 0; l < L; ++l, ++i) {
-            const lq_layer* ly = at(t, l);
-            const int b = i % nbr;
-            const char* xin = (const char*)d_x + (size_t)(M * (t * sum_k + k_before)) * esz;
-            float* yout = d_y + M * (t * sum_n + n_before);
-            st = enqueue_linear(xin, x_dtype, M, ly, t, yout, (char*)d_ws + (size_t)b * per,
-                                bs->st[b], i >= nbr, true);
-            if (st != LQ_OK) break;
-            k_before += ly->wq->K;
-            n_before += ly->wq->N;
-          }
+        std::vector<int64_t> k_before(L, 0), n_before(L, 0);
+        for (int l = 1; l < L; ++l) {
+          k_before[l] = k_before[l - 1] + at(0, l - 1)->wq->K;
+          n_before[l] = n_before[l - 1] + at(0, l - 1)->wq->N;
+        }
+        for (size_t i = 0; i < units.size() && st == LQ_OK; ++i) {
+          const Unit& u = units[i];
+          const int b = (int)(i % nbr);
+          const char* xin =
+              (const char*)d_x + (size_t)(M * (u.t * sum_k + k_before[u.l])) * esz;
+          float* yout = d_y + M * (u.t * sum_n + n_before[u.l]);
+          st = enqueue_linear(xin, x_dtype, M, at(u.t, u.l), u.t, yout,
+                              (char*)d_ws + (size_t)b * per, bs->st[b], i >= (size_t)nbr, true,
+                              u.w, M * sum_k, M * sum_n);
         }
         // join every branch back (also after an error, so no capture is left unjoined)
         for (int b = 0; b < nbr; ++b) {

@@ -389,10 +389,13 @@ cudaError_t launch_trajectory_hessian(const uint16_t* X, int64_t R, int64_t K, u
                                       const char** why);
 
 // GEMV (lq_gemv.cu)
-// qa: activation codes in the kOpGemvAct layout, asum their group sums
+// qa: activation codes in the kOpGemvAct layout, asum their group sums.
+// Rows come in segments of seg_rows (the loops of one launch): row m is written
+// at y + (m / seg_rows) * y_stride + (m % seg_rows) * N (one segment: seg_rows = M).
 cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa,
                               const uint8_t* w4, const float* sw, float* y, int64_t M, int64_t N,
-                              int64_t K, cudaStream_t s, bool pdl = false);
+                              int64_t K, cudaStream_t s, bool pdl = false,
+                              int64_t seg_rows = INT64_MAX, int64_t y_stride = 0);
 constexpr int kGemvMaxM = 16;
 
 }  // namespace lq

@@ -35,6 +35,16 @@
 namespace lq {
 namespace {
 
+// output offset of activation row m (rows in segments of seg_rows, segment
+// starts y_stride floats apart) and the extent of the rows' outputs
+__device__ __forceinline__ size_t gemv_y_offset(int m, int seg_rows, long long y_stride, int N) {
+  const int j = m / seg_rows;
+  return (size_t)j * (size_t)y_stride + (size_t)(m - j * seg_rows) * N;
+}
+__device__ __forceinline__ size_t gemv_y_extent(int M, int seg_rows, long long y_stride, int N) {
+  return gemv_y_offset(M - 1, seg_rows, y_stride, N) + N;
+}
+
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
 
@@ -56,7 +66,7 @@ template <int MB, int GPL, int RPW, bool kDB>
 __global__ void __launch_bounds__(kGemvThreads, kDB ? 1 : 3) k_group_gemv(
     const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
     const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
-    int N, int K) {
+    int N, int K, int seg_rows, long long y_stride) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   pdl_trigger();
   const int G = K / kGroup;
@@ -166,9 +176,10 @@ __global__ void __launch_bounds__(kGemvThreads, kDB ? 1 : 3) k_group_gemv(
       const int n = gw + (j0 + r) * W;
 #pragma unroll
       for (int m = 0; m < MB; ++m)
-        if (lane == ((r * MB + m) & 31) && m < M && n < N &&
-            LQ_IN_RANGE((size_t)m * N + n, (size_t)M * N))
-          y[(size_t)m * N + n] = part[r][m];
+        if (lane == ((r * MB + m) & 31) && m < M && n < N) {
+          const size_t yi = gemv_y_offset(m, seg_rows, y_stride, N) + n;
+          if (LQ_IN_RANGE(yi, gemv_y_extent(M, seg_rows, y_stride, N))) y[yi] = part[r][m];
+        }
     }
   };
 
@@ -263,7 +274,7 @@ template <int NB, int kS, int kU, int kMinBlocks>
 __global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
     const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
     const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
-    int N, int K) {
+    int N, int K, int seg_rows, long long y_stride) {
   static_assert(kU % 8 == 0 && kS >= 2, "stages of whole 8-chunk swizzle blocks, double buffered");
   constexpr int kStageW = 16 * kU * 16;  // packed codes of a stage
   constexpr int kStage = (int)mma_stage_bytes(kU);
@@ -281,6 +292,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
   const int my_rb = gw < n_rb ? (n_rb - gw + W - 1) / W : 0;
   const int n_stages = my_rb * stages_per_rb;
   const bool vec_steps = (G & 3) == 0;  // 16-byte step chunks are aligned
+  const size_t y_ext = gemv_y_extent(M, seg_rows, y_stride, N);
+  (void)y_ext;
 
   // copy stage b of this warp (row block gw + (b / stages_per_rb) * W, groups
   // (b % stages_per_rb) * kU ..) into slot b % kS; one commit group per stage
@@ -412,13 +425,15 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
 #pragma unroll
       for (int j = 0; j < NB; ++j) {
         const int m0 = j * 8 + 2 * t;
+        const size_t o0 = gemv_y_offset(m0, seg_rows, y_stride, N);
+        const size_t o1 = gemv_y_offset(m0 + 1, seg_rows, y_stride, N);
         if (na < N) {
-          if (m0 < M && LQ_IN_RANGE(na, N)) y[(size_t)m0 * N + na] = acc[j][0].x;
-          if (m0 + 1 < M && LQ_IN_RANGE(na, N)) y[(size_t)(m0 + 1) * N + na] = acc[j][0].y;
+          if (m0 < M && LQ_IN_RANGE(o0 + na, y_ext)) y[o0 + na] = acc[j][0].x;
+          if (m0 + 1 < M && LQ_IN_RANGE(o1 + na, y_ext)) y[o1 + na] = acc[j][0].y;
         }
         if (nb < N) {
-          if (m0 < M && LQ_IN_RANGE(nb, N)) y[(size_t)m0 * N + nb] = acc[j][1].x;
-          if (m0 + 1 < M && LQ_IN_RANGE(nb, N)) y[(size_t)(m0 + 1) * N + nb] = acc[j][1].y;
+          if (m0 < M && LQ_IN_RANGE(o0 + nb, y_ext)) y[o0 + nb] = acc[j][1].x;
+          if (m0 + 1 < M && LQ_IN_RANGE(o1 + nb, y_ext)) y[o1 + nb] = acc[j][1].y;
         }
         acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
       }
@@ -471,7 +486,7 @@ cudaError_t blocks_per_sm(F* k, int threads, size_t smem, size_t max_smem, int* 
 template <int MB, int GPL, int RPW, bool kDB>
 cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                        const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
-                       bool pdl) {
+                       bool pdl, int seg, long long ys) {
   const size_t smem = gemv_smem_bytes(M, K / kGroup);
   auto* k = k_group_gemv<MB, GPL, RPW, kDB>;
   int per_sm = 0;
@@ -482,24 +497,24 @@ cudaError_t launch_cfg(const int8_t* qa, const int* asum, const float* sa, const
   const int64_t want = (warps_needed + kGemvWarps - 1) / kGemvWarps;
   const int64_t blocks = std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
   return launch_kernel(k, dim3((unsigned)blocks), dim3(kGemvThreads), smem, s, pdl, qa, asum, sa,
-                       w4, sw, y, (int)M, (int)N, (int)K);
+                       w4, sw, y, (int)M, (int)N, (int)K, seg, ys);
 }
 
 // one batch per warp fits in a resident wave: no prefetch registers needed
 template <int MB, int GPL, int RPW>
 cudaError_t launch_rpw(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                        const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
-                       bool pdl) {
+                       bool pdl, int seg, long long ys) {
   const int64_t one_wave_rows = (int64_t)num_sms() * 2 * kGemvWarps * RPW;
   if (N <= one_wave_rows)
-    return launch_cfg<MB, GPL, RPW, false>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  return launch_cfg<MB, GPL, RPW, true>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+    return launch_cfg<MB, GPL, RPW, false>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
+  return launch_cfg<MB, GPL, RPW, true>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
 }
 
 template <int NB, int kS, int kU>
 cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                        const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
-                       bool pdl) {
+                       bool pdl, int seg, long long ys) {
   const int64_t G = K / kGroup;
   const size_t smem = mma_act_bytes(NB, G) + (size_t)kMmaWarps * kS * mma_stage_bytes(kU);
   if (smem > kMmaMaxSmem) return cudaErrorInvalidValue;
@@ -511,7 +526,7 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
   const int64_t want = (row_blocks + kMmaWarps - 1) / kMmaWarps;
   const int64_t blocks = std::min<int64_t>(want, (int64_t)num_sms() * per_sm);
   return launch_kernel(k, dim3((unsigned)blocks), dim3(kMmaWarps * 32), smem, s, pdl, qa, asum,
-                       sa, w4, sw, y, (int)M, (int)N, (int)K);
+                       sa, w4, sw, y, (int)M, (int)N, (int)K, seg, ys);
 }
 
 // the tensor-core GEMV for M tokens: one block of 8 tokens with 16-group
@@ -520,18 +535,18 @@ cudaError_t launch_mma(const int8_t* qa, const int* asum, const float* sa, const
 // K = 8544 at 16 tokens, above the K <= 8192 of the GEMV path
 cudaError_t launch_tc(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                       const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
-                      bool pdl) {
-  if (M <= 8) return launch_mma<1, 2, 16>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  return launch_mma<2, 3, 8>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+                      bool pdl, int seg, long long ys) {
+  if (M <= 8) return launch_mma<1, 2, 16>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
+  return launch_mma<2, 3, 8>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
 }
 
 template <int MB>
 cudaError_t launch_mb(const int8_t* qa, const int* asum, const float* sa, const uint8_t* w4,
                       const float* sw, float* y, int64_t M, int64_t N, int64_t K, cudaStream_t s,
-                      bool pdl) {
+                      bool pdl, int seg, long long ys) {
   const int64_t G = K / kGroup;
-  if (G > 128) return launch_rpw<MB, 8, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  if (G > 64) return launch_rpw<MB, 4, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  if (G > 128) return launch_rpw<MB, 8, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
+  if (G > 64) return launch_rpw<MB, 4, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
   // up to 4 tokens: when one resident wave covers N, three weight rows per warp in a single
   // batch (decode-sized launches, latency-bound); beyond that, two rows per warp
   // with the next batch in flight, the fastest streaming shape measured (a
@@ -539,33 +554,37 @@ cudaError_t launch_mb(const int8_t* qa, const int* asum, const float* sa, const 
   // with one)
   if (N >= (int64_t)num_sms() * kGemvWarps * 3 * 3 / 2) {
     if (N <= (int64_t)num_sms() * 2 * kGemvWarps * 3)
-      return launch_cfg<MB, 2, 3, false>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-    return launch_cfg<MB, 2, 2, true>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+      return launch_cfg<MB, 2, 3, false>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
+    return launch_cfg<MB, 2, 2, true>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
   }
-  return launch_rpw<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  return launch_rpw<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
 }
 
 }  // namespace
 
 cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa,
                               const uint8_t* w4, const float* sw, float* y, int64_t M, int64_t N,
-                              int64_t K, cudaStream_t s, bool pdl) {
+                              int64_t K, cudaStream_t s, bool pdl, int64_t seg_rows,
+                              int64_t y_stride) {
   if (M == 0 || N == 0) return cudaSuccess;
   if (K > (int64_t)kGroup * 32 * 8 || M > kGemvMaxM ||
-      gemv_smem_bytes(M, K / kGroup) > kGemvMaxSmem)
+      gemv_smem_bytes(M, K / kGroup) > kGemvMaxSmem || seg_rows < 1 || y_stride < 0)
     return cudaErrorInvalidValue;
+  const int seg = (int)std::min<int64_t>(seg_rows, M);
+  const long long ys = seg >= M ? 0 : (long long)y_stride;
+  if (seg < M && ys < (long long)seg * N) return cudaErrorInvalidValue;  // segments overlap
   // one token: dp4a (a 263 MB launch timed alone: 5.47 TB/s, against 5.25
   // on the tensor-core path, whose block prologue shows when launches are
   // isolated)
-  if (M <= 1) return launch_mb<1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+  if (M <= 1) return launch_mb<1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
   // 2 to 4 tokens: dp4a while the rows fit in about one resident wave of
   // warps (one memory latency per warp, the decode-sized launches); once the
   // launch streams at least a wave of 16-row blocks, the tensor-core path
   // with its deeper weight pipeline (a 263 MB launch at M = 4: 5.5 TB/s
   // against 2.9 with dp4a)
   if (M <= 4 && N < (int64_t)num_sms() * 2 * kMmaWarps * 16)
-    return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
-  return launch_tc(qa, asum, sa, w4, sw, y, M, N, K, s, pdl);
+    return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
+  return launch_tc(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
 }
 
 unsigned long long bounds_fail_gemv() { return lq_take_bounds_fail(); }
