@@ -92,6 +92,14 @@ def decode_copies(wl):
     return max(1, -(-4 * L2_BYTES // per))
 
 
+def decode_weight_passes(wl):
+    """Weight passes of one open-mode decode step: the library runs the loops of
+    a linear in one GEMV pass while their rows fit the GEMV's 16-row limit (at
+    most 8 loops per launch)."""
+    nbd = max(1, min(wl.T, 8, 16 // wl.M))
+    return -(-wl.T // nbd)
+
+
 def work_per_step(wl, copies=1):
     """Integer ops (2 per MAC) of one step and the rotation FLOPs (2 per FMA)."""
     ops = sum(2 * wl.M * lin.N * lin.K for lin in wl.linears) * wl.T * copies
@@ -457,11 +465,11 @@ def roofline_of(kernels, wl, n_probe, copies, peaks, sustained):
         peak = SM_COUNT * FP64_FMA_PER_SM_CLK * 2 * SM_CLOCK_GHZ * 1e9 / 1e12
         r = {"bound": "alu", "achieved": flops / avg_s / 1e12, "peak": peak,
              "unit": "TFLOP/s", "peak_source": "derived: 148 SM x 64 FP64 FMA/clk x 2 x 1.965 GHz"}
-    else:  # GEMV: one linear's weight stream (packed codes + steps) per launch, whatever
-        # the number of loops batched into it, plus its float32 outputs; no L2 credit
-        n_lin = len(wl.linears)
-        wbytes = sum(lin.N * lin.K * 5 // 8 for lin in wl.linears) / n_lin
-        ybytes = rows_per_launch / n_lin * sum(lin.N * 4 for lin in wl.linears) / n_lin
+    else:  # GEMV: the weight streams (packed codes + steps) of a launch, each linear
+        # once per weight pass, plus the float32 outputs; no L2 credit
+        passes = decode_weight_passes(wl)
+        wbytes = passes * sum(lin.N * lin.K * 5 // 8 for lin in wl.linears) * copies / per_step
+        ybytes = sum(wl.M * lin.N * 4 * T for lin in wl.linears) * copies / per_step
         byts = wbytes + ybytes
         r = {"bound": "hbm", "achieved": byts / avg_s / 1e9, "peak": peaks["hbm_gbs"],
              "unit": "GB/s", "peak_source": peaks["source"] + " copy bandwidth",
@@ -617,11 +625,8 @@ def measure_stack(lq, ctx, wl, n_steps, warmup, n_probe, peaks, want_clocks=Fals
     kernels = probe_kernels(lq, ctx, step, n_probe, not big) if n_probe else None
     if is_decode(wl):
         xb, wb, yb = step_bytes(wl, copies)
-        # weight passes per step: one per GEMV launch of a linear (the loops
-        # batched into a launch share its pass), counted by the probe
-        passes = wl.T
-        if kernels and "gemv" in kernels:
-            passes = kernels["gemv"]["launches"] / n_probe / (copies * len(wl.linears))
+        # weight passes per step: the loops batched into one GEMV pass share it
+        passes = decode_weight_passes(wl)
         line["weight_passes_per_step"] = passes
         line["weight_bytes_per_step"] = passes * wb
         line["weight_stream_GB_s"] = passes * wb / (ms * 1e-3) / 1e9
@@ -906,6 +911,10 @@ def run_lq(args, rank, world, local_rank):
             "aux": aux, "cpu_baseline": cpu, "e2e": e2e, "clocks": line["clocks"],
             "gpu_launches": None if launches is None else int(round(launches * args.steps)),
         }
+        if is_decode(wl):
+            out["decode"] = {k: line[k] for k in (
+                "weight_passes_per_step", "weight_bytes_per_step", "weight_stream_GB_s",
+                "weight_stream_frac_hbm", "tokens_per_s_per_linear") if k in line}
         print(json.dumps(out), flush=True)
 
 

@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cmath>
 #include <map>
+#include <memory>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -400,6 +401,28 @@ int64_t decode_branch_bytes(const std::vector<const lq_layer*>& tl, int64_t M) {
   return per;
 }
 
+// The work units of a decode-sized open-mode stack (tl: T x L handles): loops
+// t .. t + w - 1 of layer l in one quantize and one GEMV launch, w = nbd when
+// one handle serves all of those loops, else one unit per loop.
+struct DecodeUnit {
+  int t, l, w;
+};
+void decode_units(const std::vector<const lq_layer*>& tl, int L, int T, int nbd,
+                  std::vector<DecodeUnit>* units) {
+  units->clear();
+  for (int t = 0; t < T; t += nbd) {
+    const int nb = std::min(nbd, T - t);
+    for (int l = 0; l < L; ++l) {
+      bool same = true;
+      for (int j = 1; j < nb; ++j) same = same && tl[(size_t)(t + j) * L + l] == tl[(size_t)t * L + l];
+      if (same)
+        units->push_back({t, l, nb});
+      else
+        for (int j = 0; j < nb; ++j) units->push_back({t + j, l, 1});
+    }
+  }
+}
+
 lq_status check_layer_call(const lq_layer* layer, int64_t M, int32_t x_dtype) {
   if (!layer) {
     set_error("null layer");
@@ -710,11 +733,12 @@ int64_t lq_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64
   bool decode = (int64_t)T * L > 1;
   for (int i = 0; i < L; ++i) decode = decode && use_gemv(M, layers[i]->wq->K);
   const std::vector<const lq_layer*> tl(layers, layers + L);
-  if (decode) {  // one workspace slice per concurrent decode chain of loop-batched steps
+  if (decode) {  // one workspace region per unit of a grouped round (covers the chains)
     const int nbd = decode_loops_per_launch(tl, M, T);
     const int64_t units = (int64_t)((T + nbd - 1) / nbd) * L;
     need = std::max(need, decode_branch_bytes(tl, M * nbd) *
-                              std::min<int64_t>(kDecodeBranches, units));
+                              std::min<int64_t>(std::max<int64_t>(kGroupMaxUnits, kDecodeBranches),
+                                                units));
   }
   return need;
 }
@@ -766,23 +790,81 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
       // units of work: the loops t .. t + nbd - 1 of layer l in one quantize
       // and one GEMV launch (the weights streamed once for them) when the
       // same handle serves all of them, else one unit per loop
+      std::vector<DecodeUnit> units;
       int nbd = decode_loops_per_launch(tl, M, T);
-      int64_t per = decode_branch_bytes(tl, M * nbd);
-      while (nbd > 1 && ws_bytes < 2 * per) per = decode_branch_bytes(tl, M * --nbd);
-      struct Unit {
-        int t, l, w;
-      };
-      std::vector<Unit> units;
-      for (int t = 0; t < T; t += nbd) {
-        const int nb = std::min(nbd, T - t);
-        for (int l = 0; l < L; ++l) {
-          bool same = true;
-          for (int j = 1; j < nb; ++j) same = same && at(t + j, l) == at(t, l);
-          if (same)
-            units.push_back({t, l, nb});
-          else
-            for (int j = 0; j < nb; ++j) units.push_back({t + j, l, 1});
+      decode_units(tl, L, T, nbd, &units);
+      std::vector<int64_t> k_before(L, 0), n_before(L, 0);
+      for (int l = 1; l < L; ++l) {
+        k_before[l] = k_before[l - 1] + at(0, l - 1)->wq->K;
+        n_before[l] = n_before[l - 1] + at(0, l - 1)->wq->N;
+      }
+      // all units in one quantize and one GEMV launch (per round of up to
+      // kGroupMaxUnits units), when their shapes fit the grouped kernels and
+      // the workspace holds a region per unit of a round
+      {
+        const int64_t per = decode_branch_bytes(tl, M * nbd);
+        bool ok = ws_bytes >= per * std::min<int64_t>(kGroupMaxUnits, (int64_t)units.size());
+        for (const DecodeUnit& u : units) {
+          const lq_layer* ly = at(u.t, u.l);
+          ok = ok && ly->P1 != nullptr && use_gemv(M * u.w, ly->wq->K) &&
+               group_unit_ok(M * u.w, ly->wq->K, ly->a, ly->b);
         }
+        if (ok) {
+          const bool pdl = !probe_on();
+          std::unique_ptr<GroupLaunch> P(new GroupLaunch());
+          // rounds of equal size
+          const size_t n_rounds = (units.size() + kGroupMaxUnits - 1) / kGroupMaxUnits;
+          const size_t per_round = (units.size() + n_rounds - 1) / n_rounds;
+          for (size_t r0 = 0; r0 < units.size(); r0 += per_round) {
+            const int n = (int)std::min(per_round, units.size() - r0);
+            P->n_units = n;
+            for (int i = 0; i < n; ++i) {
+              const DecodeUnit& u = units[r0 + i];
+              const lq_layer* ly = at(u.t, u.l);
+              const int64_t K = ly->wq->K, rows = M * u.w;
+              GroupUnit& g = P->u[i];
+              char* reg = (char*)d_ws + (size_t)i * per;
+              g.x = (const char*)d_x + (size_t)(M * (u.t * sum_k + k_before[u.l])) * esz;
+              g.P1 = ly->P1;
+              g.P2 = ly->P2;
+              g.w4 = ly->wq->codes4;
+              g.sw = ly->wq->scales;
+              g.y = d_y + M * (u.t * sum_n + n_before[u.l]);
+              g.codes = (int8_t*)reg;
+              g.scales = (float*)(reg + round_up(rows * K, 256));
+              g.asum = (int*)((char*)g.scales + round_up(rows * (K / kGroup) * 4, 256));
+              g.x_stride = M * sum_k;
+              g.y_stride = M * sum_n;
+              for (int j = 0; j < kMaxLoopsPerLaunch; ++j)
+                g.c[j] = j < u.w ? ly->las[u.t + j] : 0.f;
+              g.K = (int)K;
+              g.N = (int)ly->wq->N;
+              g.a = ly->a;
+              g.b = ly->b;
+              g.seg_rows = (int)M;
+              g.rows = (int)rows;
+              g.qmax = ly->a_bits == 8 ? 127 : 7;
+              g.blk0 = 0;
+            }
+            cudaError_t e;
+            {
+              ProbeScope ps(kProbeRotQuant, s);
+              e = launch_quantize_units(*P, x_dtype, s, pdl && r0 > 0);
+            }
+            if (e != cudaSuccess) return cuda_error(e, "grouped quantize launch");
+            {
+              ProbeScope ps(kProbeGemv, s);
+              e = launch_gemv_units(*P, s, pdl);
+            }
+            if (e != cudaSuccess) return cuda_error(e, "grouped gemv launch");
+          }
+          return LQ_OK;
+        }
+      }
+      int64_t per = decode_branch_bytes(tl, M * nbd);
+      if (nbd > 1 && ws_bytes < 2 * per) {
+        while (nbd > 1 && ws_bytes < 2 * per) per = decode_branch_bytes(tl, M * --nbd);
+        decode_units(tl, L, T, nbd, &units);
       }
       const int nbr = (int)std::min(std::min((int64_t)kDecodeBranches, (int64_t)units.size()),
                                     ws_bytes / per);
@@ -796,13 +878,8 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
         for (int b = 0; b < nbr; ++b)
           if ((e = cudaStreamWaitEvent(bs->st[b], bs->fork, 0)) != cudaSuccess)
             return cuda_error(e, "fork wait");
-        std::vector<int64_t> k_before(L, 0), n_before(L, 0);
-        for (int l = 1; l < L; ++l) {
-          k_before[l] = k_before[l - 1] + at(0, l - 1)->wq->K;
-          n_before[l] = n_before[l - 1] + at(0, l - 1)->wq->N;
-        }
         for (size_t i = 0; i < units.size() && st == LQ_OK; ++i) {
-          const Unit& u = units[i];
+          const DecodeUnit& u = units[i];
           const int b = (int)(i % nbr);
           const char* xin =
               (const char*)d_x + (size_t)(M * (u.t * sum_k + k_before[u.l])) * esz;

@@ -398,4 +398,40 @@ cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa
                               int64_t seg_rows = INT64_MAX, int64_t y_stride = 0);
 constexpr int kGemvMaxM = 16;
 
+// ---------------------------------------------------------------------------
+// Grouped decode: the independent (layer, loop batch) units of a decode-sized
+// open-mode stack in one quantize launch and one GEMV launch.  A unit holds
+// rows = seg_rows * (loops) activation rows: row m is row m % seg_rows of loop
+// m / seg_rows, read at x + (m / seg_rows) * x_stride + (m % seg_rows) * K
+// elements and written at y + (m / seg_rows) * y_stride + (m % seg_rows) * N;
+// its activation codes (kOpGemvAct layout), steps and group sums live in its
+// own workspace region.  The table is a kernel parameter (__grid_constant__).
+// ---------------------------------------------------------------------------
+struct GroupUnit {
+  const void* x;
+  const float* P1;
+  const float* P2;
+  const uint8_t* w4;  // resident packed codes, N x K/2
+  const float* sw;    // resident steps, N x K/32
+  float* y;
+  int8_t* codes;
+  float* scales;
+  int* asum;
+  long long x_stride;  // elements between the loops' inputs
+  long long y_stride;  // floats between the loops' outputs
+  float c[kMaxLoopsPerLaunch];  // LAS clip of each loop of the unit
+  int K, N, a, b, seg_rows, rows, qmax;
+  int blk0;  // GEMV: first block of the unit (set by launch_gemv_units)
+};
+constexpr int kGroupMaxUnits = 96;  // 96 x 152 B of parameters (the limit is 32 KB)
+struct GroupLaunch {
+  GroupUnit u[kGroupMaxUnits];
+  int n_units;
+  int total_blocks;  // GEMV blocks over all units
+};
+// whether a unit's shapes fit the grouped kernels (few-row rotation, GEMV rows)
+bool group_unit_ok(int64_t rows, int64_t K, int a, int b);
+cudaError_t launch_quantize_units(const GroupLaunch& P, int x_dtype, cudaStream_t s, bool pdl);
+cudaError_t launch_gemv_units(GroupLaunch& P, cudaStream_t s, bool pdl);
+
 }  // namespace lq

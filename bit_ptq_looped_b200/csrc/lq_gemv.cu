@@ -270,26 +270,24 @@ __host__ __device__ constexpr size_t mma_act_bytes(int NB, int64_t G) {
 }
 __host__ __device__ constexpr size_t mma_stage_bytes(int kU) { return (size_t)16 * kU * (16 + 4); }
 
-template <int NB, int kS, int kU, int kMinBlocks>
-__global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
+// One block's work: warp w walks the row blocks rb_first(w), + rb_step, ...
+// (my_rb of them); all warps of the block stage the same activation.
+template <int NB, int kS, int kU>
+__device__ __forceinline__ void gemv_mma_block(
     const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
     const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
-    int N, int K, int seg_rows, long long y_stride) {
+    int N, int K, int seg_rows, long long y_stride, int rb_first, int rb_step, int my_rb,
+    unsigned char* smem_raw) {
   static_assert(kU % 8 == 0 && kS >= 2, "stages of whole 8-chunk swizzle blocks, double buffered");
   constexpr int kStageW = 16 * kU * 16;  // packed codes of a stage
   constexpr int kStage = (int)mma_stage_bytes(kU);
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  pdl_trigger();
   const int G = K / kGroup;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int gw = blockIdx.x * kMmaWarps + warp, W = gridDim.x * kMmaWarps;
   const size_t rowstride = (size_t)K / 2;
   unsigned char* ring = smem_raw + mma_act_bytes(NB, G) + (size_t)warp * kS * kStage;
   const uint32_t ring_s = smem_u32(ring);
   const int stages_per_rb = (G + kU - 1) / kU;
-  const int n_rb = (N + 15) / 16;
-  const int my_rb = gw < n_rb ? (n_rb - gw + W - 1) / W : 0;
   const int n_stages = my_rb * stages_per_rb;
   const bool vec_steps = (G & 3) == 0;  // 16-byte step chunks are aligned
   const size_t y_ext = gemv_y_extent(M, seg_rows, y_stride, N);
@@ -299,7 +297,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
   // (b % stages_per_rb) * kU ..) into slot b % kS; one commit group per stage
   auto issue = [&](int b) {
     if (b < n_stages) {
-      const int rb = gw + (b / stages_per_rb) * W, g0 = (b % stages_per_rb) * kU;
+      const int rb = rb_first + (b / stages_per_rb) * rb_step, g0 = (b % stages_per_rb) * kU;
       const uint32_t st = ring_s + (uint32_t)((b % kS) * kStage);
       const bool full = rb * 16 + 16 <= N && g0 + kU <= G;  // no row or group outside
 #pragma unroll
@@ -408,7 +406,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
     }
   };
 
-  int rb = gw, g0 = 0;
+  int rb = rb_first, g0 = 0;
   for (int b = 0; b < n_stages; ++b) {
     issue(b + kS - 1);
     cp_async_wait<kS - 1>();  // this thread's copies of stage b have landed
@@ -438,12 +436,51 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
         acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
       }
       g0 = 0;
-      rb += W;
+      rb += rb_step;
     } else {
       g0 += kU;
     }
   }
   cp_async_wait<0>();  // no copy outlives the block
+}
+
+template <int NB, int kS, int kU, int kMinBlocks>
+__global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma(
+    const int8_t* __restrict__ qa, const int* __restrict__ asum_g, const float* __restrict__ sa,
+    const uint8_t* __restrict__ w4, const float* __restrict__ sw, float* __restrict__ y, int M,
+    int N, int K, int seg_rows, long long y_stride) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5;
+  const int gw = blockIdx.x * kMmaWarps + warp, W = gridDim.x * kMmaWarps;
+  const int n_rb = (N + 15) / 16;
+  const int my_rb = gw < n_rb ? (n_rb - gw + W - 1) / W : 0;
+  gemv_mma_block<NB, kS, kU>(qa, asum_g, sa, w4, sw, y, M, N, K, seg_rows, y_stride, gw, W, my_rb,
+                             smem_raw);
+}
+
+// The grouped decode GEMV: unit u owns blocks [blk0_u, blk0_{u+1}), which split
+// its row blocks into equal contiguous ranges; the warps of a block take the
+// range's row blocks in turn.
+template <int NB, int kS, int kU, int kMinBlocks>
+__global__ void __launch_bounds__(kMmaWarps * 32, kMinBlocks) k_group_gemv_mma_units(
+    const __grid_constant__ GroupLaunch P) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  int lo = 0, hi = P.n_units - 1;  // the last unit whose first block is at or before this one
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.u[mid].blk0 <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+  }
+  const GroupUnit& U = P.u[lo];
+  const int nblk = (lo + 1 < P.n_units ? P.u[lo + 1].blk0 : P.total_blocks) - U.blk0;
+  const int j = (int)blockIdx.x - U.blk0;
+  const int n_rb = (U.N + 15) / 16;
+  const int rb0 = (int)((int64_t)n_rb * j / nblk), rb1 = (int)((int64_t)n_rb * (j + 1) / nblk);
+  const int first = rb0 + (int)(threadIdx.x >> 5);
+  const int my_rb = first < rb1 ? (rb1 - first + kMmaWarps - 1) / kMmaWarps : 0;
+  gemv_mma_block<NB, kS, kU>(U.codes, U.asum, U.scales, U.w4, U.sw, U.y, U.rows, U.N, U.K,
+                             U.seg_rows, U.y_stride, first, kMmaWarps, my_rb, smem_raw);
 }
 
 size_t gemv_smem_bytes(int64_t M, int64_t G) { return (size_t)M * G * (32 + 8); }
@@ -560,6 +597,31 @@ cudaError_t launch_mb(const int8_t* qa, const int* asum, const float* sa, const 
   return launch_rpw<MB, 2, 1>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
 }
 
+// grouped decode GEMV: units get blocks in proportion to their row blocks, one
+// resident wave over all units (at least one block per unit, at most one per
+// row block)
+template <int NB, int kS, int kU>
+cudaError_t launch_units_cfg(GroupLaunch& P, int64_t G, int64_t total_rb, cudaStream_t s,
+                             bool pdl) {
+  const size_t smem = mma_act_bytes(NB, G) + (size_t)kMmaWarps * kS * mma_stage_bytes(kU);
+  if (smem > kMmaMaxSmem) return cudaErrorInvalidValue;
+  auto* k = k_group_gemv_mma_units<NB, kS, kU, 2>;
+  int per_sm = 0;
+  cudaError_t e = blocks_per_sm(k, kMmaWarps * 32, smem, kMmaMaxSmem, &per_sm);
+  if (e != cudaSuccess) return e;
+  const int64_t slots = (int64_t)num_sms() * per_sm;
+  int64_t blk = 0;
+  for (int i = 0; i < P.n_units; ++i) {
+    const int64_t n_rb = (P.u[i].N + 15) / 16;
+    const int64_t nb = std::max<int64_t>(1, std::min(n_rb, (n_rb * slots + total_rb - 1) / total_rb));
+    P.u[i].blk0 = (int)blk;
+    blk += nb;
+  }
+  if (blk > INT32_MAX) return cudaErrorInvalidValue;
+  P.total_blocks = (int)blk;
+  return launch_kernel(k, dim3((unsigned)blk), dim3(kMmaWarps * 32), smem, s, pdl, P);
+}
+
 }  // namespace
 
 cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa,
@@ -585,6 +647,24 @@ cudaError_t launch_group_gemv(const int8_t* qa, const int* asum, const float* sa
   if (M <= 4 && N < (int64_t)num_sms() * 2 * kMmaWarps * 16)
     return launch_mb<4>(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
   return launch_tc(qa, asum, sa, w4, sw, y, M, N, K, s, pdl, seg, ys);
+}
+
+cudaError_t launch_gemv_units(GroupLaunch& P, cudaStream_t s, bool pdl) {
+  if (P.n_units <= 0) return cudaSuccess;
+  if (P.n_units > kGroupMaxUnits) return cudaErrorInvalidValue;
+  int max_rows = 0;
+  int64_t max_G = 0, total_rb = 0;
+  for (int i = 0; i < P.n_units; ++i) {
+    const GroupUnit& U = P.u[i];
+    if (U.rows < 1 || U.rows > kGemvMaxM || U.K % kGroup || U.K > kGroup * 32 * 8 || U.N < 1 ||
+        U.seg_rows < 1 || (U.rows > U.seg_rows && U.y_stride < (long long)U.seg_rows * U.N))
+      return cudaErrorInvalidValue;
+    max_rows = std::max(max_rows, U.rows);
+    max_G = std::max<int64_t>(max_G, U.K / kGroup);
+    total_rb += (U.N + 15) / 16;
+  }
+  if (max_rows <= 8) return launch_units_cfg<1, 2, 16>(P, max_G, total_rb, s, pdl);
+  return launch_units_cfg<2, 3, 8>(P, max_G, total_rb, s, pdl);
 }
 
 unsigned long long bounds_fail_gemv() { return lq_take_bounds_fail(); }

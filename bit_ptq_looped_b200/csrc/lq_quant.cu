@@ -849,19 +849,18 @@ __host__ __device__ inline SmallRotLayout small_rot_layout(int a, int b) {
   return L;
 }
 
+// One block's work: row m of the launch (input row xrow, clip c), column
+// slice sl.  With x_early the input is read before pdl_wait, which then comes
+// before the first store (a previous kernel may still read the output
+// buffers); without it the caller has waited already.
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
-    const Tin* __restrict__ x, int K, const float* __restrict__ P1, int a,
-    const float* __restrict__ P2, int b, const LoopSegs segs, int qmax,
-    int8_t* __restrict__ codes8, int opf, uint8_t* __restrict__ codes4,
-    float* __restrict__ scales, int* __restrict__ asum, int x_early) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  pdl_trigger();
-  if (!x_early) pdl_wait();
+__device__ __forceinline__ void rotate_quant_small_block(
+    const Tin* __restrict__ xrow, int K, const float* __restrict__ P1, int a,
+    const float* __restrict__ P2, int b, float c, int qmax, int8_t* __restrict__ codes8, int opf,
+    uint8_t* __restrict__ codes4, float* __restrict__ scales, int* __restrict__ asum,
+    int x_early, int m, int sl, unsigned char* smem_raw) {
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr int kWarps = kThreads / 32;
-  const int S = b >> 5;
-  const int m = blockIdx.x / S, sl = blockIdx.x - m * S;
   const SmallRotLayout L = small_rot_layout(a, b);
   double* P2T = reinterpret_cast<double*>(smem_raw + L.off_p2t);
   double* P1T = reinterpret_cast<double*>(smem_raw + L.off_p1t);
@@ -871,12 +870,6 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
   const FastDiv fd_b((uint32_t)b), fd_a((uint32_t)a);
 
   // ---- loads, all of a thread's in flight together
-  const int64_t jseg = (int64_t)m / segs.seg_rows;
-  const Tin* xrow = x + jseg * segs.x_stride + ((int64_t)m - jseg * segs.seg_rows) * K;
-  float c = segs.c[0];  // static indices keep the parameter block out of local memory
-#pragma unroll
-  for (int u = 1; u < kMaxLoopsPerLaunch; ++u)
-    if (jseg == u) c = segs.c[u];
   {
     constexpr int kP2U = kSmallMaxB * 32 / kThreads, kP1U = kSmallMaxA * kSmallMaxA / kThreads;
     constexpr int kXU = kSmallMaxA * kSmallMaxB / 8 / kThreads;
@@ -970,6 +963,46 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
       store_codes<false>(q, st, chunk, codes8, opf, codes4, scales);
     }
   }
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
+    const Tin* __restrict__ x, int K, const float* __restrict__ P1, int a,
+    const float* __restrict__ P2, int b, const LoopSegs segs, int qmax,
+    int8_t* __restrict__ codes8, int opf, uint8_t* __restrict__ codes4,
+    float* __restrict__ scales, int* __restrict__ asum, int x_early) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  if (!x_early) pdl_wait();
+  const int S = b >> 5;
+  const int m = blockIdx.x / S, sl = blockIdx.x - m * S;
+  const int64_t jseg = (int64_t)m / segs.seg_rows;
+  const Tin* xrow = x + jseg * segs.x_stride + ((int64_t)m - jseg * segs.seg_rows) * K;
+  float c = segs.c[0];  // static indices keep the parameter block out of local memory
+#pragma unroll
+  for (int u = 1; u < kMaxLoopsPerLaunch; ++u)
+    if (jseg == u) c = segs.c[u];
+  rotate_quant_small_block<Tin>(xrow, K, P1, a, P2, b, c, qmax, codes8, opf, codes4, scales,
+                                asum, x_early, m, sl, smem_raw);
+}
+
+// The grouped decode quantizer: block (x, y) is block x of unit y (row
+// x / S, slice x % S of the unit's rows; blocks past the unit's rows exit).
+// The inputs were written before the sequence began.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) k_rotate_quant_small_units(
+    const __grid_constant__ GroupLaunch P) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  const GroupUnit& U = P.u[blockIdx.y];
+  const int S = U.b >> 5;
+  if ((int)blockIdx.x >= U.rows * S) return;
+  const int m = blockIdx.x / S, sl = blockIdx.x - m * S;
+  const int jseg = m / U.seg_rows;
+  const Tin* xrow = static_cast<const Tin*>(U.x) + (int64_t)jseg * U.x_stride +
+                    (int64_t)(m - jseg * U.seg_rows) * U.K;
+  rotate_quant_small_block<Tin>(xrow, U.K, U.P1, U.a, U.P2, U.b, U.c[jseg], U.qmax, U.codes,
+                                kOpGemvAct, nullptr, U.scales, U.asum, 1, m, sl, smem_raw);
 }
 
 
@@ -1192,6 +1225,36 @@ cudaError_t launch_weight_operand(const uint8_t* codes4, const float* sw, int64_
                        codes4, n_words, opf, op, sw, N, G, sw_t, n_conv);
 }
 
+
+bool group_unit_ok(int64_t rows, int64_t K, int a, int b) {
+  return rows >= 1 && rows <= kSmallRotMaxRows && K <= 8192 && (int64_t)a * b == K &&
+         b % 32 == 0 && a <= kSmallMaxA && b <= kSmallMaxB;
+}
+
+cudaError_t launch_quantize_units(const GroupLaunch& P, int x_dtype, cudaStream_t s, bool pdl) {
+  if (P.n_units <= 0) return cudaSuccess;
+  if (P.n_units > kGroupMaxUnits) return cudaErrorInvalidValue;
+  int max_blocks = 0;
+  size_t ssm = 0;
+  for (int i = 0; i < P.n_units; ++i) {
+    const GroupUnit& U = P.u[i];
+    if (!group_unit_ok(U.rows, U.K, U.a, U.b) || U.seg_rows < 1 ||
+        (U.rows + U.seg_rows - 1) / U.seg_rows > kMaxLoopsPerLaunch)
+      return cudaErrorInvalidValue;
+    max_blocks = std::max(max_blocks, U.rows * (U.b / 32));
+    ssm = std::max(ssm, small_rot_layout(U.a, U.b).bytes);
+  }
+  const dim3 grid((unsigned)max_blocks, (unsigned)P.n_units);
+  cudaError_t e;
+  if (x_dtype == LQ_BF16) {
+    auto* k = k_rotate_quant_small_units<__nv_bfloat16>;
+    if ((e = set_smem(k, ssm)) != cudaSuccess) return e;
+    return launch_kernel(k, grid, dim3(kThreads), ssm, s, pdl, P);
+  }
+  auto* k = k_rotate_quant_small_units<float>;
+  if ((e = set_smem(k, ssm)) != cudaSuccess) return e;
+  return launch_kernel(k, grid, dim3(kThreads), ssm, s, pdl, P);
+}
 
 unsigned long long bounds_fail_quant() { return lq_take_bounds_fail(); }
 

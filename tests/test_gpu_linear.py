@@ -257,15 +257,15 @@ def test_loop_stack_open_batching_matches_per_loop(wl, M):
 
 @pytest.mark.parametrize("M,a_bits", [(1, 8), (3, 4), (4, 4), (16, 8)])
 def test_loop_stack_open_decode_branches(M, a_bits):
-    """Decode-sized open mode: the loops of a layer run in one quantize and one
-    GEMV launch while their rows fit the GEMV path (all 4 loops at 1, 3 and 4
-    tokens, one loop at 16), and those units run as concurrent chains on
-    internal streams, each with its own workspace slice.  Three linears of
-    different widths (the last with a ragged N), T = 4: every output against
-    the oracle, for the branched schedule, for the one-chain schedule a
-    minimal workspace gives (one launch per loop), and for a workspace sized
-    for one linear at T * M rows (fewer chains, smaller loop batches); the
-    branched schedule is deterministic (bit-identical on a second call)."""
+    """Decode-sized open mode: the loops of a layer form one unit while their
+    rows fit the GEMV path (all 4 loops at 1, 3 and 4 tokens, one loop at 16).
+    With the stack's workspace size every unit runs in one grouped quantize and
+    one grouped GEMV launch; a workspace for one linear at T * M rows runs the
+    units as two concurrent quantize->GEMV chains on internal streams (smaller
+    loop batches), and a minimal workspace as one chain of one launch pair per
+    loop.  Three linears of different widths (the last with a ragged N),
+    T = 4: every output of all three schedules against the oracle, and the
+    grouped schedule deterministic (bit-identical on a second call)."""
     lins = (synth.Linear("d0", 2048, 2048, 32, 64, 0), synth.Linear("d1", 2048, 5632, 32, 64, 0),
             synth.Linear("d2", 2048, 1000, 32, 64, 1))
     wl = synth.Workload(f"decode_stack_M{M}", M=M, T=4, linears=lins, a_bits=a_bits,
@@ -282,7 +282,9 @@ def test_loop_stack_open_decode_branches(M, a_bits):
     y = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, ws=ws_all)
     y1 = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, ws=ws_one)
     y2 = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, ws=ws_all, y=torch.empty_like(y))
-    # one linear at T * M rows: two chains of half-size loop batches
+    # one linear at T * M rows: two chains of half-size loop batches (at 16
+    # tokens this size, taken by the tensor-core path's operand, holds the
+    # grouped schedule's regions)
     ws_seq = lq.workspace(layers, M * wl.T)
     ys = lq.lq_loop_stack(xd, layers, wl.T, lq.LQ_OPEN, M=M, ws=ws_seq)
     torch.cuda.synchronize()
@@ -304,6 +306,58 @@ def test_loop_stack_open_decode_branches(M, a_bits):
                     quant[(t, l)] = (host(q8), host(s))
                 q8h, sh = quant[(t, l)]
                 linear_parity(yg, xs[t][l], built[l][1], t, q8h, sh, built[l][0].w_flips)
+
+
+@pytest.mark.parametrize("M,T,copies,a_bits,x_dtype", [
+    (5, 4, 1, 8, "bf16"),    # loop batches of 3 and 1 (15 and 5 rows) in one launch
+    (2, 4, 1, 4, "f32"),     # 8 rows: one token block
+    (16, 4, 9, 8, "bf16"),   # 108 units of one loop: two rounds of 54
+])
+def test_loop_stack_open_decode_grouped(M, T, copies, a_bits, x_dtype):
+    """Decode-sized open mode with the stack's own workspace size: every
+    (layer, loop batch) unit of a round in one quantize launch and one GEMV
+    launch (two launches per round, counted by the probe), each unit with its
+    own rows (ragged loop batches share a launch), layers of different widths
+    including a ragged N; every output of every loop against the oracle."""
+    lins = (synth.Linear("g0", 512, 256, 16, 32, 0), synth.Linear("g1", 2048, 1000, 32, 64, 1),
+            synth.Linear("g2", 1024, 96, 32, 32, 2))
+    wl = synth.Workload(f"decode_grouped_M{M}", M=M, T=T, linears=lins, a_bits=a_bits,
+                        outlier_frac=0.02, outlier_mult=20.0, x_dtype=x_dtype,
+                        description="grouped decode stack")
+    params = synth.module_params(wl)
+    built = [make_layer(mp, a_bits) for mp in params]
+    # the stack repeats the three linears `copies` times (same handles)
+    L = 3 * copies
+    layers = [built[l % 3][0] for l in range(L)]
+    xs = [[synth.loop_input(wl, lins[l % 3], t, rows=np.arange(M) + M * (l // 3))
+           for l in range(L)] for t in range(T)]
+    flat = np.concatenate([xs[t][l].ravel() for t in range(T) for l in range(L)])
+    xd = act_tensor(flat, x_dtype)
+    ws = lq.workspace(layers, M, T=T)
+    nbd = max(1, min(T, 8, 16 // M))
+    n_units = -(-T // nbd) * L
+    rounds = -(-n_units // 96)
+    lq.lq_probe_enable(True)
+    try:
+        y = lq.lq_loop_stack(xd, layers, T, lq.LQ_OPEN, M=M, ws=ws)
+        torch.cuda.synchronize()
+        probe = lq.lq_probe_read()
+    finally:
+        lq.lq_probe_enable(False)
+    assert probe["rotate_quantize"][1] == rounds and probe["gemv"][1] == rounds, probe
+    yh = host(y)
+    off = 0
+    for t in range(T):
+        for l in range(L):
+            lin, mp = lins[l % 3], params[l % 3]
+            n = M * lin.N
+            yg = yh[off:off + n].reshape(M, lin.N)
+            off += n
+            q8, _, s = lq.lq_quantize_act(act_tensor(xs[t][l], x_dtype), dev(mp.P1),
+                                          dev(mp.P2), float(mp.las[t]), a_bits)
+            torch.cuda.synchronize()
+            linear_parity(yg, xs[t][l], built[l % 3][1], t, host(q8), host(s),
+                          built[l % 3][0].w_flips)
 
 
 def test_loop_stack_open_more_than_eight_loops():
