@@ -423,7 +423,7 @@ struct GroupUnit {
   int K, N, a, b, seg_rows, rows, qmax;
   int blk0;  // GEMV: first block of the unit (set by launch_gemv_units)
 };
-constexpr int kGroupMaxUnits = 96;  // 96 x 152 B of parameters (the limit is 32 KB)
+constexpr int kGroupMaxUnits = 96;  // 96 x 152 B of parameters (the limit is 32764 B)
 struct GroupLaunch {
   GroupUnit u[kGroupMaxUnits];
   int n_units;

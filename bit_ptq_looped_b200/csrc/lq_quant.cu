@@ -332,16 +332,16 @@ template <> struct RawChunk<__nv_bfloat16> {
 
 constexpr int kRotTM = 2, kRotTN = 2;  // warp task: 16 x 16 outputs (measured best of 1-4 x 2-4)
 
+// The row tiles tile0, tile0 + tile_step, ... (R rows each) of one launch's
+// rows; the caller has waited for its predecessor unless x_early.
 template <typename Tin, bool kStoreF32>
-__global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
+__device__ __forceinline__ void rotate_quant_tiles(
     const Tin* __restrict__ x, int64_t M, int K, const float* __restrict__ P1, int a,
-    const float* __restrict__ P2, int b, int R, const LoopSegs segs, int qmax,
+    const float* __restrict__ P2, int b, int R, const LoopSegs& segs, int qmax,
     int8_t* __restrict__ codes8,
     int opf, uint8_t* __restrict__ codes4, float* __restrict__ scales,
-    float* __restrict__ out_f32, int* __restrict__ asum, int x_early) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  pdl_trigger();
-  if (!x_early) pdl_wait();
+    float* __restrict__ out_f32, int* __restrict__ asum, int x_early, int64_t tile0,
+    int64_t tile_step, unsigned char* smem_raw) {
   bool waited = !x_early;
   const RotLayout L = rot_layout(a, b, R);
   double* sm = reinterpret_cast<double*>(smem_raw);
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
       }
     }
   };
-  if (x_pre) prefetch_tile((int64_t)blockIdx.x * R);
+  if (x_pre) prefetch_tile(tile0 * R);
   {
     const int n2 = b * b, nf = n2 + a * a;
     for (int base = 0; base < nf; base += kFU * kThreads) {
@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
   const FastDiv fd_s1ctq((uint32_t)s1_ctq), fd_s2tok((uint32_t)(s2_rt * s1_ctq));
 
   int par = 0;
-  for (int64_t m0 = (int64_t)blockIdx.x * R; m0 < M; m0 += (int64_t)gridDim.x * R, par ^= 1) {
+  for (int64_t m0 = tile0 * R; m0 < M; m0 += tile_step * R, par ^= 1) {
     const int rows = (M - m0 < (int64_t)R) ? (int)(M - m0) : R;
     if (tid < rows) {
       const int64_t r = m0 + tid, j = r / segs.seg_rows;
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
     }
     __syncthreads();
     // the next tile's input is in flight during this tile's MMA stages
-    if (x_pre && m0 + (int64_t)gridDim.x * R < M) prefetch_tile(m0 + (int64_t)gridDim.x * R);
+    if (x_pre && m0 + tile_step * R < M) prefetch_tile(m0 + tile_step * R);
     // ---- stage 1: Y[(r,i), j] = sum_q X[(r,i), q] P2[q, j]  -> YT[r][j][i]
     for (int task = warp; task < s1_tasks; task += kWarps) {
       const int rt = (int)fd_s1ctq.div((uint32_t)task), cq = task - rt * s1_ctq;
@@ -536,6 +536,42 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
       }
     }
   }
+}
+
+template <typename Tin, bool kStoreF32>
+__global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
+    const Tin* __restrict__ x, int64_t M, int K, const float* __restrict__ P1, int a,
+    const float* __restrict__ P2, int b, int R, const LoopSegs segs, int qmax,
+    int8_t* __restrict__ codes8,
+    int opf, uint8_t* __restrict__ codes4, float* __restrict__ scales,
+    float* __restrict__ out_f32, int* __restrict__ asum, int x_early) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  if (!x_early) pdl_wait();
+  rotate_quant_tiles<Tin, kStoreF32>(x, M, K, P1, a, P2, b, R, segs, qmax, codes8, opf, codes4,
+                                     scales, out_f32, asum, x_early, blockIdx.x, gridDim.x,
+                                     smem_raw);
+}
+
+// The grouped decode quantizer: block (x, y) takes row tile x (R rows) of
+// unit y; blocks past the unit's tiles exit.  The inputs were written before
+// the sequence began.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads, 2) k_rotate_quant_units(
+    const __grid_constant__ GroupLaunch P, int R) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_trigger();
+  const GroupUnit& U = P.u[blockIdx.y];
+  const int64_t tiles = (U.rows + R - 1) / R;
+  if ((int64_t)blockIdx.x >= tiles) return;
+  LoopSegs segs;
+  segs.seg_rows = U.seg_rows;
+  segs.x_stride = U.x_stride;
+#pragma unroll
+  for (int u = 0; u < kMaxLoopsPerLaunch; ++u) segs.c[u] = U.c[u];
+  rotate_quant_tiles<Tin, false>(static_cast<const Tin*>(U.x), U.rows, U.K, U.P1, U.a, U.P2,
+                                 U.b, R, segs, U.qmax, U.codes, kOpGemvAct, nullptr, U.scales,
+                                 nullptr, U.asum, 1, blockIdx.x, tiles, smem_raw);
 }
 
 // ---------------------------------------------------------------------------
@@ -986,26 +1022,6 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
                                 asum, x_early, m, sl, smem_raw);
 }
 
-// The grouped decode quantizer: block (x, y) is block x of unit y (row
-// x / S, slice x % S of the unit's rows; blocks past the unit's rows exit).
-// The inputs were written before the sequence began.
-template <typename Tin>
-__global__ void __launch_bounds__(kThreads) k_rotate_quant_small_units(
-    const __grid_constant__ GroupLaunch P) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  pdl_trigger();
-  const GroupUnit& U = P.u[blockIdx.y];
-  const int S = U.b >> 5;
-  if ((int)blockIdx.x >= U.rows * S) return;
-  const int m = blockIdx.x / S, sl = blockIdx.x - m * S;
-  const int jseg = m / U.seg_rows;
-  const Tin* xrow = static_cast<const Tin*>(U.x) + (int64_t)jseg * U.x_stride +
-                    (int64_t)(m - jseg * U.seg_rows) * U.K;
-  rotate_quant_small_block<Tin>(xrow, U.K, U.P1, U.a, U.P2, U.b, U.c[jseg], U.qmax, U.codes,
-                                kOpGemvAct, nullptr, U.scales, U.asum, 1, m, sl, smem_raw);
-}
-
-
 // The tensor-core GEMM's weight operand, expanded from the resident packed
 // codes for one launch: blocks [0, n_conv) turn packed words (8 codes) into
 // 8 code bytes (E4M3 or int8, as the GEMM's kind reads them); blocks from
@@ -1227,33 +1243,40 @@ cudaError_t launch_weight_operand(const uint8_t* codes4, const float* sw, int64_
 
 
 bool group_unit_ok(int64_t rows, int64_t K, int a, int b) {
-  return rows >= 1 && rows <= kSmallRotMaxRows && K <= 8192 && (int64_t)a * b == K &&
-         b % 32 == 0 && a <= kSmallMaxA && b <= kSmallMaxB;
+  int R = 0;
+  return rows >= 1 && rows <= kGemvMaxM && K <= 8192 && (int64_t)a * b == K &&
+         rotate_smem_bytes(a, b, &R) > 0;
 }
 
 cudaError_t launch_quantize_units(const GroupLaunch& P, int x_dtype, cudaStream_t s, bool pdl) {
   if (P.n_units <= 0) return cudaSuccess;
   if (P.n_units > kGroupMaxUnits) return cudaErrorInvalidValue;
-  int max_blocks = 0;
-  size_t ssm = 0;
+  // one row-tile height for the launch: the smallest any unit's factors need
+  int R = 16, max_tiles = 0;
   for (int i = 0; i < P.n_units; ++i) {
     const GroupUnit& U = P.u[i];
+    int Ru = 0;
     if (!group_unit_ok(U.rows, U.K, U.a, U.b) || U.seg_rows < 1 ||
         (U.rows + U.seg_rows - 1) / U.seg_rows > kMaxLoopsPerLaunch)
       return cudaErrorInvalidValue;
-    max_blocks = std::max(max_blocks, U.rows * (U.b / 32));
-    ssm = std::max(ssm, small_rot_layout(U.a, U.b).bytes);
+    rotate_smem_bytes(U.a, U.b, &Ru);
+    R = std::min(R, Ru);
   }
-  const dim3 grid((unsigned)max_blocks, (unsigned)P.n_units);
+  size_t smem = 0;
+  for (int i = 0; i < P.n_units; ++i) {
+    smem = std::max(smem, rot_layout(P.u[i].a, P.u[i].b, R).bytes);
+    max_tiles = std::max(max_tiles, (P.u[i].rows + R - 1) / R);
+  }
+  const dim3 grid((unsigned)max_tiles, (unsigned)P.n_units);
   cudaError_t e;
   if (x_dtype == LQ_BF16) {
-    auto* k = k_rotate_quant_small_units<__nv_bfloat16>;
-    if ((e = set_smem(k, ssm)) != cudaSuccess) return e;
-    return launch_kernel(k, grid, dim3(kThreads), ssm, s, pdl, P);
+    auto* k = k_rotate_quant_units<__nv_bfloat16>;
+    if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+    return launch_kernel(k, grid, dim3(kThreads), smem, s, pdl, P, R);
   }
-  auto* k = k_rotate_quant_small_units<float>;
-  if ((e = set_smem(k, ssm)) != cudaSuccess) return e;
-  return launch_kernel(k, grid, dim3(kThreads), ssm, s, pdl, P);
+  auto* k = k_rotate_quant_units<float>;
+  if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+  return launch_kernel(k, grid, dim3(kThreads), smem, s, pdl, P, R);
 }
 
 unsigned long long bounds_fail_quant() { return lq_take_bounds_fail(); }
