@@ -144,6 +144,39 @@ def test_fused_rotate_quantize_many_rows(ab, M, x_dtype):
             np.testing.assert_array_equal(O.unpack_int4(host(q4)), host(q8))
 
 
+@pytest.mark.parametrize("M", [3, 2368 + 37])
+@pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
+def test_fused_rotate_quantize_extreme_exponents(M, x_dtype):
+    """Inputs whose float->double widening takes every path: a row of
+    subnormals only, rows mixing signed zeros and subnormals into normal
+    values, a row near 1e30 and a row near 1e-30 (few rows: the per-row
+    kernel; many: the warp-specialised one); every code against the oracle."""
+    a, b = 32, 64
+    K = a * b
+    rng = np.random.default_rng(M + 7)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[0] = (rng.standard_normal(K) * 1e-39).astype(np.float32)  # subnormal
+    x[1, ::3] = 0.0
+    x[1, 1::3] = -0.0
+    x[1, 2::7] = np.float32(3e-41)
+    x[2] *= np.float32(1e30)
+    if M > 3:
+        x[3] *= np.float32(1e-30)
+        x[4:, 5::11] = -0.0
+        x[4:, 9::13] = np.float32(-2e-40)
+    if x_dtype == "bf16":
+        x = synth.round_bf16(x)
+    assert np.any((x != 0) & (np.abs(x) < np.finfo(np.float32).tiny))
+    P1, P2 = _orthogonal(a, 41), _orthogonal(b, 42)
+    xt64 = O.kron_rotate_f64(x, P1, P2)
+    for bits in (4, 8):
+        q8, _, s = lq.lq_quantize_act(act_tensor(x, x_dtype), dev(P1), dev(P2), 0.85, bits)
+        torch.cuda.synchronize()
+        q_or, s_or = O.quantize_groups(xt64.astype(np.float32), 0.85, bits)
+        flips = check_codes_near_tie(host(q8), host(s), q_or, s_or, xt64)
+        assert len(flips) == 0
+
+
 def test_fused_rotation_identity_factors_reduce_to_plain_rtn():
     M, K = 100, 2048
     x = _outlier_matrix(M, K, seed=3)
