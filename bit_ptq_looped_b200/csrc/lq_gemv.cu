@@ -293,32 +293,43 @@ __device__ __forceinline__ void gemv_mma_block(
   const size_t y_ext = gemv_y_extent(M, seg_rows, y_stride, N);
   (void)y_ext;
 
-  // copy stage b of this warp (row block gw + (b / stages_per_rb) * W, groups
+  // copy stage b of this warp (row block rb_first + (b / stages_per_rb) * rb_step, groups
   // (b % stages_per_rb) * kU ..) into slot b % kS; one commit group per stage
+  // the stage issued next: its row block and first group (calls come in stage
+  // order, so they advance by one stage each, without a division)
+  int is_rb = rb_first, is_g0 = 0;
   auto issue = [&](int b) {
     if (b < n_stages) {
-      const int rb = rb_first + (b / stages_per_rb) * rb_step, g0 = (b % stages_per_rb) * kU;
+      const int rb = is_rb, g0 = is_g0;
+      if (g0 + kU >= G) {
+        is_g0 = 0;
+        is_rb += rb_step;
+      } else {
+        is_g0 += kU;
+      }
       const uint32_t st = ring_s + (uint32_t)((b % kS) * kStage);
       const bool full = rb * 16 + 16 <= N && g0 + kU <= G;  // no row or group outside
+      const uint8_t* wb = w4 + (size_t)rb * 16 * rowstride + (size_t)g0 * 16;
+      const float* sb = sw + (size_t)rb * 16 * G + g0;
 #pragma unroll
       for (int i = 0; i < kU / 2; ++i) {
         const int c = lane + 32 * i, r = c / kU, u = c % kU;
-        const int n = rb * 16 + r, grp = g0 + u;
-        if (full || (n < N && grp < G))
+        if (full || (rb * 16 + r < N && g0 + u < G))
           cp_async16(st + (uint32_t)((r * kU + (u ^ (r & 7))) * 16),
-                     w4 + (size_t)n * rowstride + (size_t)grp * 16);
+                     wb + (uint32_t)(r * (int)rowstride + u * 16));
       }
 #pragma unroll
       for (int i = 0; i < kU / 8; ++i) {
         const int c = lane + 32 * i, r = c / (kU / 4), h = c % (kU / 4), n = rb * 16 + r;
         const int grp = g0 + 4 * h;
         const uint32_t dst = st + kStageW + (uint32_t)(r * kU * 4 + h * 16);
+        const float* src = sb + (uint32_t)(r * G + 4 * h);
         if (vec_steps) {
-          if (n < N && grp < G) cp_async16(dst, sw + (size_t)n * G + grp);
+          if (n < N && grp < G) cp_async16(dst, src);
         } else {
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (n < N && grp + e < G) cp_async4(dst + 4 * e, sw + (size_t)n * G + grp + e);
+            if (n < N && grp + e < G) cp_async4(dst + 4 * e, src + e);
         }
       }
     }
