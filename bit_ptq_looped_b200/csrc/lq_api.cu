@@ -142,10 +142,11 @@ bool use_gemv(int64_t M, int64_t K) {
 }
 
 // workspace: codes (M x K bytes), steps (M x G fp32), and for the GEMV path the
-// per-group code sums (M x G int32)
+// per-group code sums (M x G int32) and 256 bytes for the persistent chain
+// kernel's grid barrier
 int64_t ws_bytes_for(int64_t M, int64_t K) {
   const int64_t steps = round_up(M * (K / kGroup) * 4, 256);
-  return round_up(M * K, 256) + steps + (use_gemv(M, K) ? steps : 0);
+  return round_up(M * K, 256) + steps + (use_gemv(M, K) ? steps + 256 : 0);
 }
 
 // the GEMM's weight operand in the workspace: N x K code bytes, then the
@@ -238,7 +239,8 @@ enum ProbeKind {
   kProbeQuant = 1,
   kProbeGemm = 2,
   kProbeGemv = 3,
-  kProbeWeightOp = 4
+  kProbeWeightOp = 4,
+  kProbeChain = 5
 };
 
 struct ProbeScope {
@@ -922,6 +924,71 @@ static lq_status enqueue_stack(const void* d_x, int32_t x_dtype, int64_t M,
     }
     return LQ_OK;
   }
+  // decode-sized chain mode without CTA: every step in one persistent kernel
+  // (launches of up to kChainMaxSteps steps)
+  if (!cta && (int64_t)T * L > 1) {
+    bool ok = true;
+    size_t act = 0, fac = 0, wts = 0;
+    int64_t kmax = 0;
+    for (const lq_layer* ly : tl) {
+      size_t a1 = 0, f1 = 0, w1 = 0;
+      ok = ok && ly->P1 != nullptr && use_gemv(M, ly->wq->K) &&
+           chain_decode_ok((int)M, (int)ly->wq->K, (int)ly->wq->N, ly->a, ly->b, &a1, &f1, &w1);
+      act = std::max(act, a1);
+      fac = std::max(fac, f1);
+      wts = std::max(wts, w1);
+      kmax = std::max(kmax, ly->wq->K);
+    }
+    const size_t smem = act + fac + wts;
+    if (ok && smem <= 220u * 1024u && ws_bytes >= ws_bytes_for(M, kmax)) {
+      std::unique_ptr<ChainLaunch> P(new ChainLaunch());
+      const int64_t steps_b = round_up(M * (kmax / kGroup) * 4, 256);
+      P->M = (int)M;
+      P->act_bytes = (int)act;
+      P->fac_bytes = (int)fac;
+      P->codes = (int8_t*)d_ws;
+      P->scales = (float*)((char*)d_ws + round_up(M * kmax, 256));
+      P->asum = (int*)((char*)P->scales + steps_b);
+      P->bar = (unsigned*)((char*)P->asum + steps_b);
+      float* yc = d_y;
+      const void* xin = d_x;
+      bool x_bf16 = x_dtype == LQ_BF16;
+      int n = 0;
+      for (int t = 0; t < T; ++t) {
+        for (int l = 0; l < L; ++l) {
+          const lq_layer* ly = at(t, l);
+          ChainStep& c = P->s[n++];
+          c.x = xin;
+          c.P1 = ly->P1;
+          c.P2 = ly->P2;
+          c.w4 = ly->wq->codes4;
+          c.sw = ly->wq->scales;
+          c.y = yc;
+          c.c = ly->las[t];
+          c.K = (int)ly->wq->K;
+          c.N = (int)ly->wq->N;
+          c.a = ly->a;
+          c.b = ly->b;
+          c.qmax = ly->a_bits == 8 ? 127 : 7;
+          c.x_bf16 = x_bf16 ? 1 : 0;
+          xin = yc;
+          x_bf16 = false;
+          yc += M * ly->wq->N;
+          if (n == kChainMaxSteps || (t == T - 1 && l == L - 1)) {
+            P->n_steps = n;
+            cudaError_t e;
+            {
+              ProbeScope ps(kProbeChain, s);
+              e = launch_chain_decode(*P, smem, s);
+            }
+            if (e != cudaSuccess) return cuda_error(e, "chain decode launch");
+            n = 0;
+          }
+        }
+      }
+      return LQ_OK;
+    }
+  }
   float* ycur = d_y;
   const float* prev_y = nullptr;
   // CTA state (the adapted input of the next loop) after the codes and steps
@@ -1340,6 +1407,21 @@ lq_status lq_selftest_bounded_wait(int64_t limit_us, void* stream) {
     return LQ_ERR_ARG;
   }
   cudaError_t e = launch_wait_selftest((uint64_t)limit_us * 1000u, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_error(e, "self-test launch");
+  return LQ_OK;
+}
+
+lq_status lq_selftest_grid_wait(int64_t limit_us, void* d_scratch, void* stream) {
+  if (limit_us <= 0 || limit_us > 10000000) {
+    set_error("limit must be in (0, 10 s]");
+    return LQ_ERR_ARG;
+  }
+  if (!d_scratch || (uintptr_t)d_scratch % 4) {
+    set_error("scratch must be 8 bytes of 4-byte aligned device memory");
+    return LQ_ERR_ARG;
+  }
+  cudaError_t e = launch_grid_wait_selftest((uint64_t)limit_us * 1000u, (cudaStream_t)stream,
+                                            (unsigned*)d_scratch);
   if (e != cudaSuccess) return cuda_error(e, "self-test launch");
   return LQ_OK;
 }

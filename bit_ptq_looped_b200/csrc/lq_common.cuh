@@ -200,6 +200,28 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// cp.async copies into shared memory (one commit group per call of commit)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+// sum of four products of unsigned bytes (a) and signed bytes (b), plus c
+__device__ __forceinline__ int dp4a_us(uint32_t a_unsigned, uint32_t b_signed, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a_unsigned), "r"(b_signed), "r"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -429,6 +451,44 @@ struct GroupLaunch {
   int n_units;
   int total_blocks;  // GEMV blocks over all units
 };
+// ---------------------------------------------------------------------------
+// Chain-mode decode in one persistent kernel: the steps of a chain-mode stack
+// (each step's input the previous step's output) with grid barriers between
+// the few-row quantize and the GEMV of each step.  The table is a kernel
+// parameter; `work` is the step's activation region (codes in the kOpGemvAct
+// layout, steps, group sums) followed by the barrier's two words.
+// ---------------------------------------------------------------------------
+struct ChainStep {
+  const void* x;   // M x K input rows (the stack's input, else the previous output)
+  const float* P1;
+  const float* P2;
+  const uint8_t* w4;  // resident packed codes, N x K/2
+  const float* sw;    // resident steps, N x K/32
+  float* y;           // M x N output
+  float c;            // LAS clip of the step's loop
+  int K, N, a, b, qmax, x_bf16;
+};
+constexpr int kChainMaxSteps = 128;  // 128 x 80 B of parameters
+struct ChainLaunch {
+  ChainStep s[kChainMaxSteps];
+  int n_steps, M;
+  int act_bytes, fac_bytes;  // shared-memory regions: rotation / activation, raw factors
+  int8_t* codes;
+  float* scales;
+  int* asum;
+  unsigned* bar;  // two words, zeroed before the launch
+};
+// whether a step's shapes fit the persistent kernel (its shared memory and the
+// few-row rotation), and the step's shared-memory regions: rotation scratch /
+// activation, raw factors, weight rows (the launch takes the maximum of each)
+bool chain_decode_ok(int M, int K, int N, int a, int b, size_t* act, size_t* fac, size_t* wts);
+cudaError_t launch_chain_decode(const ChainLaunch& P, size_t smem, cudaStream_t s);
+// the persistent kernel's status word (LQ_ERR_DEVICE_TIMEOUT after a grid
+// barrier gave up), read and cleared
+int take_chain_status();
+// diagnostic: a grid barrier that one block never reaches, bounded by limit_ns
+cudaError_t launch_grid_wait_selftest(uint64_t limit_ns, cudaStream_t s, unsigned* bar);
+
 // whether a unit's shapes fit the grouped kernels (few-row rotation, GEMV rows)
 bool group_unit_ok(int64_t rows, int64_t K, int a, int b);
 cudaError_t launch_quantize_units(const GroupLaunch& P, int x_dtype, cudaStream_t s, bool pdl);

@@ -739,7 +739,13 @@ lq_status read_and_clear_device_status(cudaStream_t s) {
   if (v != 0) {
     e = cudaMemcpyToSymbol(g_gemm_status, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_error(e, "clear device status");
+    take_chain_status();  // one report covers both status words
     set_error("a bounded device-side wait expired in the GEMM kernel (status %d)", v);
+    return (lq_status)v;
+  }
+  v = take_chain_status();
+  if (v != 0) {
+    set_error("a grid barrier of the persistent decode kernel gave up (status %d)", v);
     return (lq_status)v;
   }
   return LQ_OK;

@@ -299,14 +299,17 @@ __device__ __forceinline__ void load_row_chunk8(const Tin* __restrict__ x, int64
   d[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-// 8 input elements held as raw vectors, so a prefetch does not wait for its data
+// 8 input elements held as raw vectors, so a prefetch does not wait for its data.
+// kCg: load through L2 only (data the same kernel wrote on another SM), else
+// through the read-only path (data written before the kernel started).
 template <typename Tin> struct RawChunk;
 template <> struct RawChunk<float> {
   float4 v0, v1;
+  template <bool kCg = false>
   __device__ __forceinline__ void load(const float* __restrict__ x, int64_t chunk) {
     const float4* p = reinterpret_cast<const float4*>(x + chunk * 8);
-    v0 = __ldg(p);
-    v1 = __ldg(p + 1);
+    v0 = kCg ? __ldcg(p) : __ldg(p);
+    v1 = kCg ? __ldcg(p + 1) : __ldg(p + 1);
   }
   __device__ __forceinline__ void zero() { v0 = v1 = make_float4(0.f, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ void store(float* dst) const {
@@ -316,8 +319,10 @@ template <> struct RawChunk<float> {
 };
 template <> struct RawChunk<__nv_bfloat16> {
   uint4 v;
+  template <bool kCg = false>
   __device__ __forceinline__ void load(const __nv_bfloat16* __restrict__ x, int64_t chunk) {
-    v = __ldg(reinterpret_cast<const uint4*>(x + chunk * 8));
+    const uint4* p = reinterpret_cast<const uint4*>(x + chunk * 8);
+    v = kCg ? __ldcg(p) : __ldg(p);
   }
   __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
   __device__ __forceinline__ void store(float* dst) const {
@@ -553,9 +558,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant(
                                      smem_raw);
 }
 
-// The grouped decode quantizer: block (x, y) takes row tile x (R rows) of
-// unit y; blocks past the unit's tiles exit.  The inputs were written before
-// the sequence began.
+// The grouped decode quantizer: block (x, y) takes row tiles x, x + gridDim.x,
+// ... (R rows each) of unit y, staging the unit's factors once; blocks past
+// the unit's tiles exit.  The inputs were written before the sequence began.
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant_units(
     const __grid_constant__ GroupLaunch P, int R) {
@@ -571,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_rotate_quant_units(
   for (int u = 0; u < kMaxLoopsPerLaunch; ++u) segs.c[u] = U.c[u];
   rotate_quant_tiles<Tin, false>(static_cast<const Tin*>(U.x), U.rows, U.K, U.P1, U.a, U.P2,
                                  U.b, R, segs, U.qmax, U.codes, kOpGemvAct, nullptr, U.scales,
-                                 nullptr, U.asum, 1, blockIdx.x, tiles, smem_raw);
+                                 nullptr, U.asum, 1, blockIdx.x, gridDim.x, smem_raw);
 }
 
 // ---------------------------------------------------------------------------
@@ -888,13 +893,14 @@ __host__ __device__ inline SmallRotLayout small_rot_layout(int a, int b) {
 // One block's work: row m of the launch (input row xrow, clip c), column
 // slice sl.  With x_early the input is read before pdl_wait, which then comes
 // before the first store (a previous kernel may still read the output
-// buffers); without it the caller has waited already.
-template <typename Tin>
+// buffers); without it the caller has waited already.  kCg: the input was
+// written by the same kernel (read through L2, not the read-only path).
+template <typename Tin, bool kCg = false>
 __device__ __forceinline__ void rotate_quant_small_block(
     const Tin* __restrict__ xrow, int K, const float* __restrict__ P1, int a,
     const float* __restrict__ P2, int b, float c, int qmax, int8_t* __restrict__ codes8, int opf,
     uint8_t* __restrict__ codes4, float* __restrict__ scales, int* __restrict__ asum,
-    int x_early, int m, int sl, unsigned char* smem_raw) {
+    int x_early, int m, int sl, unsigned char* smem_raw, bool factors_ready = false) {
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr int kWarps = kThreads / 32;
   const SmallRotLayout L = small_rot_layout(a, b);
@@ -914,16 +920,17 @@ __device__ __forceinline__ void rotate_quant_small_block(
     RawChunk<Tin> xv[kXU];
 #pragma unroll
     for (int u = 0; u < kXU; ++u)
-      if (u * kThreads + tid < nx) xv[u].load(xrow, u * kThreads + tid);
+      if (u * kThreads + tid < nx) xv[u].template load<kCg>(xrow, u * kThreads + tid);
 #pragma unroll
     for (int u = 0; u < kP2U; ++u) {  // element (q, j) = (e / 32, e % 32) of the slice
       const int e = u * kThreads + tid;
-      p2v[u] = e < n2 ? __ldg(P2 + (size_t)(e >> 5) * b + 32 * sl + (e & 31)) : 0.f;
+      p2v[u] = e < n2 && !factors_ready ? __ldg(P2 + (size_t)(e >> 5) * b + 32 * sl + (e & 31))
+                                        : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < kP1U; ++u) {
       const int e = u * kThreads + tid;
-      p1v[u] = e < n1 ? __ldg(P1 + e) : 0.f;
+      p1v[u] = e < n1 && !factors_ready ? __ldg(P1 + e) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < kXU; ++u) {
@@ -933,17 +940,19 @@ __device__ __forceinline__ void rotate_quant_small_block(
         xv[u].store(Xs + (size_t)i * L.ldx + q);
       }
     }
+    if (!factors_ready) {
 #pragma unroll
-    for (int u = 0; u < kP2U; ++u) {
-      const int e = u * kThreads + tid;
-      if (e < n2) P2T[(size_t)(e & 31) * L.ldp2 + (e >> 5)] = (double)p2v[u];
-    }
+      for (int u = 0; u < kP2U; ++u) {
+        const int e = u * kThreads + tid;
+        if (e < n2) P2T[(size_t)(e & 31) * L.ldp2 + (e >> 5)] = (double)p2v[u];
+      }
 #pragma unroll
-    for (int u = 0; u < kP1U; ++u) {
-      const int e = u * kThreads + tid;
-      if (e < n1) {
-        const int pp = (int)fd_a.div((uint32_t)e), i = e - pp * a;
-        P1T[(size_t)i * L.ldp1 + pp] = (double)p1v[u];
+      for (int u = 0; u < kP1U; ++u) {
+        const int e = u * kThreads + tid;
+        if (e < n1) {
+          const int pp = (int)fd_a.div((uint32_t)e), i = e - pp * a;
+          P1T[(size_t)i * L.ldp1 + pp] = (double)p1v[u];
+        }
       }
     }
   }
@@ -1020,6 +1029,276 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
     if (jseg == u) c = segs.c[u];
   rotate_quant_small_block<Tin>(xrow, K, P1, a, P2, b, c, qmax, codes8, opf, codes4, scales,
                                 asum, x_early, m, sl, smem_raw);
+}
+
+// ---------------------------------------------------------------------------
+// Chain-mode decode: one persistent kernel over the steps of a stack.
+//
+// One block per SM (a cooperative launch, so every block is resident and a
+// wait never depends on a block that has not started).  Per step:
+//  1. every block starts copying its slice of the step's weights (rows
+//     [n0, n1) of N: packed codes and steps, both contiguous in memory) into
+//     shared memory with cp.async, not waited for yet;
+//  2. blocks 0 .. M * b/32 - 1 stage their factors, wait until every block
+//     has written the previous step's output (a counter of blocks), then
+//     rotate and quantize one (row, 32-column slice) of the step's input each
+//     (the few-row block above), write the activation codes (kOpGemvAct
+//     layout), steps and group sums, and count themselves done;
+//  3. every block waits for the step's quantize blocks (a second counter),
+//     copies the activation into shared memory, waits for its weight rows
+//     and forms y[m][n] for them: warp per weight row, lane per group, dp4a
+//     on the offset-binary nibbles minus 8 * sum q_a, the fold with both
+//     steps in float32, a butterfly sum over the lanes per token (the same
+//     arithmetic, in the same order, as the dp4a GEMV kernel), and counts
+//     itself done.
+// Only the blocks that need a result wait for it; the counters only grow
+// within a launch (zeroed before it), so no reset races a waiter.  A wait
+// gives up after limit_ns: the block records LQ_ERR_DEVICE_TIMEOUT, drains
+// its copies and returns, and every other waiter then gives up at once.
+// ---------------------------------------------------------------------------
+__device__ int g_chain_status = 0;
+constexpr int kChainMaxM = 4;
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Step counters in global memory (zeroed before the launch): a block signals
+// after its stores (block barrier, then one thread's fence and atomic add),
+// and a block waits until a counter reaches a target (one thread's acquire
+// loads, then a block barrier).  A wait gives up after limit_ns, or at once
+// when another block already has; false then.
+// (the block barrier orders the block's stores before thread 0's release add,
+// and thread 0's acquire load before the block's loads after the barrier)
+__device__ __forceinline__ void chain_signal(unsigned* cnt) {
+  __syncthreads();
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(cnt) : "memory");
+}
+
+__device__ bool chain_wait(const unsigned* cnt, unsigned target, uint64_t limit_ns) {
+  __shared__ int ok;
+  if (threadIdx.x == 0) {
+    ok = 1;
+    if ((int)(ld_acquire_u32(cnt) - target) < 0) {
+      const uint64_t t0 = global_timer_ns();
+      while ((int)(ld_acquire_u32(cnt) - target) < 0) {
+        if (*(volatile int*)&g_chain_status != 0 || global_timer_ns() - t0 > limit_ns) {
+          atomicExch(&g_chain_status, (int)LQ_ERR_DEVICE_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  return ok != 0;
+}
+
+// The few-row block's factors: P2's 32-column slice sl (b rows of 32 floats)
+// and P1 (a x a), copied raw into `fsm` by cp.async ahead of their step (one
+// commit group, possibly empty, per call), then widened into the block's
+// float64 operands in shared memory.
+__host__ __device__ inline size_t chain_fac_bytes(int a, int b) {
+  return ((size_t)b * 32 + (size_t)a * a) * sizeof(float);
+}
+__device__ __forceinline__ void chain_issue_factors(const ChainStep& S, int sl, bool mine,
+                                                    unsigned char* fsm) {
+  if (mine) {
+    const int n2 = S.b * 8, n1 = S.a * S.a / 4;  // 16-byte chunks
+    for (int i = threadIdx.x; i < n2; i += kThreads) {
+      const int q = i >> 3, c = i & 7;
+      cp_async16(smem_u32(fsm + 16 * (size_t)i), S.P2 + (size_t)q * S.b + 32 * sl + 4 * c);
+    }
+    for (int i = threadIdx.x; i < n1; i += kThreads)
+      cp_async16(smem_u32(fsm + (size_t)S.b * 128 + 16 * (size_t)i), S.P1 + 4 * (size_t)i);
+  }
+  cp_async_commit();
+}
+__device__ __forceinline__ void chain_widen_factors(int a, int b, const unsigned char* fsm,
+                                                    unsigned char* smem_raw) {
+  const SmallRotLayout L = small_rot_layout(a, b);
+  double* P2T = reinterpret_cast<double*>(smem_raw + L.off_p2t);
+  double* P1T = reinterpret_cast<double*>(smem_raw + L.off_p1t);
+  const float* p2 = reinterpret_cast<const float*>(fsm);
+  const float* p1 = p2 + (size_t)b * 32;
+  const FastDiv fd_a((uint32_t)a);
+  for (int e = threadIdx.x; e < b * 32; e += kThreads)
+    P2T[(size_t)(e & 31) * L.ldp2 + (e >> 5)] = (double)p2[e];
+  for (int e = threadIdx.x; e < a * a; e += kThreads) {
+    const int pp = (int)fd_a.div((uint32_t)e), i = e - pp * a;
+    P1T[(size_t)i * L.ldp1 + pp] = (double)p1[e];
+  }
+}
+
+__host__ __device__ inline size_t chain_act_bytes(int M, int K, int a, int b) {
+  const size_t act = (size_t)M * K + 2 * (size_t)M * (K / kGroup) * 4;
+  const size_t rot = small_rot_layout(a, b).bytes;
+  return ((act > rot ? act : rot) + 15) & ~(size_t)15;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_chain_decode(const __grid_constant__ ChainLaunch P,
+                                                                uint64_t limit_ns) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int kWarps = kThreads / 32;
+  const int M = P.M;
+  // shared memory: rotation scratch, later the activation | raw factors | weights, their steps
+  unsigned char* fsm = smem_raw + P.act_bytes;
+  unsigned char* wsm = fsm + P.fac_bytes;
+  auto q_slice = [&](int st) {  // this block's slice in step st's quantize, or -1
+    const int Sl = P.s[st].b >> 5;
+    return (int)blockIdx.x < M * Sl ? (int)blockIdx.x % Sl : -1;
+  };
+  chain_issue_factors(P.s[0], q_slice(0), q_slice(0) >= 0, fsm);
+  unsigned q_target = 0;  // quantize blocks of the steps so far
+  for (int s = 0; s < P.n_steps; ++s) {
+    const ChainStep& S = P.s[s];
+    const int K = S.K, N = S.N, G = K / kGroup;
+    const int n0 = (int)((int64_t)N * blockIdx.x / gridDim.x);
+    const int n1 = (int)((int64_t)N * (blockIdx.x + 1) / gridDim.x);
+    const int rows = n1 - n0;
+    float* swsm = reinterpret_cast<float*>(wsm + (size_t)rows * (K / 2));
+    {  // this block's weight rows of the step (pending groups: factors, weights)
+      const int n_w = rows * (K / 32), n_s = rows * G / 4;  // 16-byte chunks
+      const uint8_t* wsrc = S.w4 + (size_t)n0 * (K / 2);
+      const float* ssrc = S.sw + (size_t)n0 * G;
+      for (int i = tid; i < n_w; i += kThreads) cp_async16(smem_u32(wsm + 16 * (size_t)i), wsrc + 16 * (size_t)i);
+      for (int i = tid; i < n_s; i += kThreads) cp_async16(smem_u32(swsm + 4 * (size_t)i), ssrc + 4 * (size_t)i);
+      cp_async_commit();
+    }
+    // ---- quantize the step's input: its factors (copied during the previous
+    // step) widened first, then, once every block has written the previous
+    // step's output, the input rows
+    const int Sl = S.b >> 5;
+    q_target += (unsigned)(M * Sl);
+    const int sl = q_slice(s);
+    if (sl >= 0) {
+      const int m = (int)blockIdx.x / Sl;
+      cp_async_wait<1>();  // the factors (the weights may still be in flight)
+      __syncthreads();
+      chain_widen_factors(S.a, S.b, fsm, smem_raw);
+      if (s > 0 && !chain_wait(P.bar + 1, (unsigned)s * gridDim.x, limit_ns)) {
+        cp_async_wait<0>();
+        return;
+      }
+      if (S.x_bf16)
+        rotate_quant_small_block<__nv_bfloat16, true>(
+            static_cast<const __nv_bfloat16*>(S.x) + (size_t)m * K, K, S.P1, S.a, S.P2, S.b, S.c,
+            S.qmax, P.codes, kOpGemvAct, nullptr, P.scales, P.asum, 0, m, sl, smem_raw, true);
+      else
+        rotate_quant_small_block<float, true>(static_cast<const float*>(S.x) + (size_t)m * K, K,
+                                              S.P1, S.a, S.P2, S.b, S.c, S.qmax, P.codes,
+                                              kOpGemvAct, nullptr, P.scales, P.asum, 0, m, sl,
+                                              smem_raw, true);
+      chain_signal(P.bar);
+    }
+    // the next step's factors (pending groups: weights, next factors); the
+    // rotation above has finished reading this step's
+    if (s + 1 < P.n_steps) chain_issue_factors(P.s[s + 1], q_slice(s + 1), q_slice(s + 1) >= 0, fsm);
+    // ---- every quantize block of this step has written its codes
+    if (!chain_wait(P.bar, q_target, limit_ns)) {
+      cp_async_wait<0>();
+      return;
+    }
+    // ---- the GEMV of this block's weight rows
+    uint4* act = reinterpret_cast<uint4*>(smem_raw);              // M * 2 * G vectors
+    int* asum = reinterpret_cast<int*>(act + (size_t)M * 2 * G);  // M * G
+    float* ssa = reinterpret_cast<float*>(asum + (size_t)M * G);  // M * G
+    {
+      // written by other blocks of this kernel: loads through L2
+      const uint4* src = reinterpret_cast<const uint4*>(P.codes);
+      for (int i = tid; i < M * 2 * G; i += kThreads) act[i] = __ldcg(src + i);
+      for (int i = tid; i < M * G; i += kThreads) {
+        asum[i] = __ldcg(P.asum + i);
+        ssa[i] = __ldcg(P.scales + i);
+      }
+    }
+    if (s + 1 < P.n_steps)
+      cp_async_wait<1>();  // the weights (the next factors may still be in flight)
+    else
+      cp_async_wait<0>();
+    __syncthreads();
+    // two weight rows per warp at a time: r0 = 2 * warp, + 2 * kWarps, ...
+    for (int r0 = 2 * warp; r0 < rows; r0 += 2 * kWarps) {
+      const bool two = r0 + 1 < rows;
+      float part[2][kChainMaxM];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int m = 0; m < kChainMaxM; ++m) part[h][m] = 0.f;
+      for (int g = lane; g < G; g += 32) {
+        uint32_t lo[2][4], hi[2][4];
+        float swg[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = two ? r0 + h : r0;
+          const uint4 w = reinterpret_cast<const uint4*>(wsm + (size_t)r * (K / 2))[g];
+          const uint32_t wu[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u,
+                                  w.w ^ 0x88888888u};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            lo[h][i] = wu[i] & 0x0F0F0F0Fu;
+            hi[h][i] = (wu[i] >> 4) & 0x0F0F0F0Fu;
+          }
+          swg[h] = swsm[(size_t)r * G + g];
+        }
+#pragma unroll
+        for (int m = 0; m < kChainMaxM; ++m) {
+          if (m < M) {
+            const uint4 a0 = act[gemv_act_vec_index(m, 0, g, G)];
+            const uint4 a1 = act[gemv_act_vec_index(m, 1, g, G)];
+            const int corr = 8 * asum[m * G + g];
+            const float sam = ssa[m * G + g];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              int d = dp4a_us(lo[h][0], a0.x, 0);
+              d = dp4a_us(hi[h][0], a0.y, d);
+              d = dp4a_us(lo[h][1], a0.z, d);
+              d = dp4a_us(hi[h][1], a0.w, d);
+              d = dp4a_us(lo[h][2], a1.x, d);
+              d = dp4a_us(hi[h][2], a1.y, d);
+              d = dp4a_us(lo[h][3], a1.z, d);
+              d = dp4a_us(hi[h][3], a1.w, d);
+              part[h][m] = fmaf(sam * swg[h], (float)(d - corr), part[h][m]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int m = 0; m < kChainMaxM; ++m) {
+          float v = part[h][m];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+          part[h][m] = v;
+        }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = n0 + r0 + h;
+        if (h == 0 || two) {
+#pragma unroll
+          for (int m = 0; m < kChainMaxM; ++m)
+            if (lane == m && m < M && LQ_IN_RANGE((size_t)m * N + n, (size_t)M * N))
+              S.y[(size_t)m * N + n] = part[h][m];
+        }
+      }
+    }
+    chain_signal(P.bar + 1);  // this block's rows of the step's output are written
+  }
+  cp_async_wait<0>();
+}
+
+// a step-counter wait that nothing satisfies
+__global__ void k_grid_wait_selftest(unsigned* bar, uint64_t limit_ns) {
+  if (threadIdx.x == 0) {
+    bar[0] = 0u;
+    bar[1] = 0u;
+  }
+  __syncthreads();
+  chain_wait(bar, 1u, limit_ns);
 }
 
 // The tensor-core GEMM's weight operand, expanded from the resident packed
@@ -1267,7 +1546,10 @@ cudaError_t launch_quantize_units(const GroupLaunch& P, int x_dtype, cudaStream_
     smem = std::max(smem, rot_layout(P.u[i].a, P.u[i].b, R).bytes);
     max_tiles = std::max(max_tiles, (P.u[i].rows + R - 1) / R);
   }
-  const dim3 grid((unsigned)max_tiles, (unsigned)P.n_units);
+  // about one resident wave (two blocks per SM) over all units: each block
+  // stages its unit's factors once and takes several of its tiles
+  const int per_unit = std::max(1, std::min(max_tiles, (2 * num_sms() + P.n_units - 1) / P.n_units));
+  const dim3 grid((unsigned)per_unit, (unsigned)P.n_units);
   cudaError_t e;
   if (x_dtype == LQ_BF16) {
     auto* k = k_rotate_quant_units<__nv_bfloat16>;
@@ -1277,6 +1559,57 @@ cudaError_t launch_quantize_units(const GroupLaunch& P, int x_dtype, cudaStream_
   auto* k = k_rotate_quant_units<float>;
   if ((e = set_smem(k, smem)) != cudaSuccess) return e;
   return launch_kernel(k, grid, dim3(kThreads), smem, s, pdl, P, R);
+}
+
+bool chain_decode_ok(int M, int K, int N, int a, int b, size_t* act, size_t* fac, size_t* wts) {
+  if (M < 1 || M > kChainMaxM || K % 128 || K > 8192 || N < 1 || (int64_t)a * b != K ||
+      b % 32 || a % 4 || a > kSmallMaxA || b > kSmallMaxB || M * (b / 32) > num_sms())
+    return false;
+  const int G = K / kGroup;
+  const size_t rows_max = (size_t)(N + num_sms() - 1) / num_sms();
+  *act = chain_act_bytes(M, K, a, b);
+  *fac = chain_fac_bytes(a, b);
+  *wts = rows_max * (K / 2 + (size_t)G * 4);
+  return *act + *fac + *wts <= 220u * 1024u;
+}
+
+cudaError_t launch_chain_decode(const ChainLaunch& P, size_t smem, cudaStream_t s) {
+  if (P.n_steps <= 0) return cudaSuccess;
+  if (P.n_steps > kChainMaxSteps || P.M < 1 || P.M > kChainMaxM || P.act_bytes % 16 ||
+      P.fac_bytes % 16 || smem > 220u * 1024u)
+    return cudaErrorInvalidValue;
+  cudaError_t e = set_smem(k_chain_decode, smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_chain_decode, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  e = cudaMemsetAsync(P.bar, 0, 2 * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)num_sms());
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint64_t limit_ns = 200ull * 1000 * 1000;  // 200 ms per barrier
+  return cudaLaunchKernelEx(&cfg, k_chain_decode, P, limit_ns);
+}
+
+int take_chain_status() {
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_chain_status, sizeof(int)) != cudaSuccess) return (int)LQ_ERR_CUDA;
+  if (v != 0) cudaMemcpyToSymbol(g_chain_status, &zero, sizeof(int));
+  return v;
+}
+
+cudaError_t launch_grid_wait_selftest(uint64_t limit_ns, cudaStream_t s, unsigned* bar) {
+  k_grid_wait_selftest<<<1, 32, 0, s>>>(bar, limit_ns);
+  return cudaGetLastError();
 }
 
 unsigned long long bounds_fail_quant() { return lq_take_bounds_fail(); }

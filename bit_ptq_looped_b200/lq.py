@@ -62,12 +62,13 @@ SIGNATURES = {
     "lq_loop_stack_cta": (_i32, [_vp, _i32, _i64, _pp, _i32, _i32, _vp, _vp, _vp, _i64, _vp]),
     "lq_check_device": (_i32, [_vp]),
     "lq_selftest_bounded_wait": (_i32, [_i64, _vp]),
+    "lq_selftest_grid_wait": (_i32, [_i64, _vp, _vp]),
     "lq_loop_linear_noalloc": (_i32, [_vp, _i32, _i64, _vp, _i32, _vp, _vp]),
     "lq_probe_enable": (_i32, [_i32]),
     "lq_probe_read": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]),
 }
 
-PROBE_KINDS = ("rotate_quantize", "quantize", "gemm", "gemv", "weight_operand")
+PROBE_KINDS = ("rotate_quantize", "quantize", "gemm", "gemv", "weight_operand", "chain_decode")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -471,3 +472,11 @@ def lq_probe_read() -> dict:
 
 def lq_selftest_bounded_wait(limit_us: int = 1000, stream=None) -> None:
     _check(lib().lq_selftest_bounded_wait(limit_us, _stream(stream)), "lq_selftest_bounded_wait")
+
+
+def lq_selftest_grid_wait(scratch: torch.Tensor, limit_us: int = 1000, stream=None) -> None:
+    """scratch: at least 8 bytes of device memory for the barrier's two words."""
+    if scratch.numel() * scratch.element_size() < 8:
+        raise ValueError("scratch needs 8 bytes")
+    _check(lib().lq_selftest_grid_wait(limit_us, _dev(scratch, "scratch"), _stream(stream)),
+           "lq_selftest_grid_wait")

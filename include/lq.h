@@ -354,10 +354,11 @@ lq_status lq_loop_linear_noalloc(const void* d_x, int32_t x_dtype, int64_t M,
  * milliseconds and the number of launches, then clears them.  Kinds (index):
  * 0 fused rotate+quantize, 1 quantize-only, 2 tensor-core GEMM, 3 GEMV,
  * 4 weight-operand expansion (the GEMM's 8-bit weight bytes and transposed
- * steps, one per GEMM launch).
+ * steps, one per GEMM launch), 5 persistent chain-mode decode (one launch
+ * covers up to 128 quantize -> GEMV steps of a decode-sized chain-mode stack).
  * h_ms and h_count point to arrays of LQ_PROBE_KINDS entries (host memory).
  */
-#define LQ_PROBE_KINDS 5
+#define LQ_PROBE_KINDS 6
 lq_status lq_probe_enable(int32_t on);
 lq_status lq_probe_read(double* h_ms, int64_t* h_count);
 
@@ -381,6 +382,16 @@ lq_status lq_check_device(void* stream);
  * usable.  A following lq_check_device(stream) reports (and clears) it.
  */
 lq_status lq_selftest_bounded_wait(int64_t limit_us, void* stream);
+
+/*
+ * lq_selftest_grid_wait -- the same diagnostic for the grid barrier of the
+ * persistent chain-mode decode kernel: one block waits at a grid barrier that
+ * expects one block more than the launch has.  The wait gives up after
+ * limit_us microseconds (0 < limit_us <= 10 s) and records
+ * LQ_ERR_DEVICE_TIMEOUT; a following lq_check_device(stream) reports (and
+ * clears) it.  d_scratch: 8 bytes of device memory the barrier uses.
+ */
+lq_status lq_selftest_grid_wait(int64_t limit_us, void* d_scratch, void* stream);
 
 #ifdef __cplusplus
 }

@@ -30,3 +30,18 @@ def test_selftest_rejects_bad_limits():
         with pytest.raises(lq.LQError) as e:
             lq.lq_selftest_bounded_wait(bad)
         assert e.value.status == lq.LQ_ERR_ARG
+
+
+def test_grid_barrier_times_out_and_reports():
+    """The persistent decode kernel's grid barrier, waiting for a block that
+    never arrives, gives up after its limit and records the timeout."""
+    lq.lq_check_device()
+    scratch = torch.zeros(2, dtype=torch.int32, device="cuda")
+    lq.lq_selftest_grid_wait(scratch, 2000)  # 2 ms limit
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_check_device()
+    assert e.value.status == lq.LQ_ERR_DEVICE_TIMEOUT
+    lq.lq_check_device()  # cleared
+    with pytest.raises(lq.LQError) as e:
+        lq.lq_selftest_grid_wait(scratch, 0)
+    assert e.value.status == lq.LQ_ERR_ARG

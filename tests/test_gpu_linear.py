@@ -470,6 +470,58 @@ def test_loop_stack_chain_tiny():
                    what=f"chain t={t}")
 
 
+def _chain_decode_case(M, a_bits, x_dtype, T):
+    """Three chained linears 2048 -> 1024 -> 3072 -> 2048 (factors 32x64,
+    32x32, 32x96), T loops with their own clips; returns the built layers,
+    the first input and the GPU outputs of the chain-mode stack with the probe
+    counts."""
+    lins = (synth.Linear("c0", 2048, 1024, 32, 64, 0), synth.Linear("c1", 1024, 3072, 32, 32, 1),
+            synth.Linear("c2", 3072, 2048, 32, 96, 2))
+    wl = synth.Workload(f"chain_M{M}", M=M, T=T, linears=lins, a_bits=a_bits,
+                        outlier_frac=0.02, outlier_mult=20.0, x_dtype=x_dtype,
+                        description="chain-mode decode stack")
+    params = synth.module_params(wl)
+    rng = np.random.default_rng(M + T)
+    for mp in params:
+        mp.las = rng.uniform(0.7, 1.0, T).astype(np.float32)
+    built = [make_layer(mp, a_bits) for mp in params]
+    x0 = synth.loop_input(wl, lins[0], 0)
+    lq.lq_probe_enable(True)
+    try:
+        y = lq.lq_loop_stack(act_tensor(x0, x_dtype), [b[0] for b in built], T, lq.LQ_CHAIN, M=M)
+        torch.cuda.synchronize()
+        probe = lq.lq_probe_read()
+    finally:
+        lq.lq_probe_enable(False)
+    return lins, params, built, x0, host(y), probe
+
+
+@pytest.mark.parametrize("M,a_bits,x_dtype,T", [(1, 8, "bf16", 4), (3, 4, "f32", 4),
+                                                (4, 8, "bf16", 4), (4, 4, "bf16", 43)])
+def test_loop_stack_chain_decode_persistent(M, a_bits, x_dtype, T):
+    """Decode-sized chain mode runs every step in the persistent kernel (one
+    launch per 128 steps, grid barriers between each step's quantize and GEMV):
+    each step's output against the oracle applied to the step's actual input
+    (the stack's input, then the previous step's float32 output)."""
+    lins, params, built, x0, y, probe = _chain_decode_case(M, a_bits, x_dtype, T)
+    L = len(lins)
+    n_launch = -(-(T * L) // 128)
+    assert probe["chain_decode"][1] == n_launch and probe["gemv"][1] == 0, probe
+    off = 0
+    xin, xin_dtype = x0, x_dtype
+    for t in range(T):
+        for l in range(L):
+            lin, mp = lins[l], params[l]
+            n = M * lin.N
+            yg = y[off:off + n].reshape(M, lin.N)
+            off += n
+            q8, _, s = lq.lq_quantize_act(act_tensor(xin, xin_dtype), dev(mp.P1), dev(mp.P2),
+                                          float(mp.las[t]), a_bits)
+            torch.cuda.synchronize()
+            linear_parity(yg, xin, built[l][1], t, host(q8), host(s), built[l][0].w_flips)
+            xin, xin_dtype = yg, "f32"
+
+
 def test_loop_stack_chain_shape_check():
     wl = synth.MLP
     params = synth.module_params(wl)
