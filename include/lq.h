@@ -171,7 +171,8 @@ void lq_layer_free(lq_layer* layer);
  * through the given layers: the activation codes and steps of one step, and
  * for the tensor-core path (M > 16) the weight operand of the largest layer
  * (N x K code bytes + G x N steps), expanded from the resident 4-bit codes by
- * each call.
+ * each call; for the GEMV path (M <= 16) the codes' group sums and 256 bytes
+ * for the step counters of the persistent chain-mode decode kernel.
  */
 int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M);
 
@@ -179,10 +180,12 @@ int64_t lq_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M);
  * Workspace with which lq_loop_stack in LQ_OPEN mode runs up to min(T, 8)
  * loops of each layer in one quantize and one GEMM launch (the loops of a
  * layer are independent in open mode and share the resident weights).  For
- * decode-sized M (the GEMV path, M <= 16) it is the size that lets the
- * independent (t, l) steps of open mode run as up to 16 concurrent
- * quantize->GEMV chains, each with its own slice (smaller workspaces run
- * fewer chains, one at least).
+ * decode-sized M (the GEMV path, M <= 16) the loops of a layer form one unit
+ * while their rows fit the GEMV (16 rows), and it is the size that gives
+ * every unit of a round (up to 96 units) its own region, so that each round
+ * runs as one grouped quantize and one grouped GEMV launch; smaller
+ * workspaces run the units as up to 16 concurrent quantize->GEMV chains on
+ * internal streams, or as one chain.
  * Returns -1 on a null pointer or a non-positive L or T.
  */
 int64_t lq_stack_workspace_bytes(const lq_layer* const* layers, int32_t L, int64_t M,
@@ -210,9 +213,13 @@ lq_status lq_loop_linear(const void* d_x, int32_t x_dtype, int64_t M, const lq_l
  *         In LQ_OPEN mode a larger workspace lets one launch cover several
  *         loops of a layer (as many as fit, at most 8;
  *         lq_stack_workspace_bytes gives the size for min(T, 8)), or, for
- *         decode-sized M, lets up to 16 (t, l) steps run concurrently on
- *         internal streams forked from and joined back into `stream`;
- *         results are the same either way.
+ *         decode-sized M, lets all units run in grouped launches or up to 16
+ *         of them concurrently on internal streams forked from and joined
+ *         back into `stream`; every schedule meets the same tolerances.
+ * In LQ_CHAIN mode a decode-sized stack (M <= 4, factors whose b is a
+ * multiple of 32, a <= 64, b <= 128, K a multiple of 128) runs all its steps
+ * in one persistent cooperative kernel per 128 steps, its waits bounded (an
+ * expired wait is reported by lq_check_device as LQ_ERR_DEVICE_TIMEOUT).
  * Consecutive kernels of the schedule use programmatic dependent launch: a
  * kernel starts its prologue (weight loads, rotation of inputs that exist
  * before the call) while its predecessor finishes, and waits for it before
