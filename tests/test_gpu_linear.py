@@ -444,6 +444,55 @@ def test_loop_stack_slt_chain_tiny():
                    what=f"slt chain t={t}")
 
 
+@pytest.mark.parametrize("mode", ["open", "chain"])
+def test_loop_stack_slt_decode(mode):
+    """SLT serving at decode size (4 tokens, two 2048 x 2048 modules, T = 4,
+    module 0 selected with its own transform and weight per loop): open mode
+    runs every unit (the selected module one loop per unit, the shared one all
+    four loops in one) in one grouped quantize and one grouped GEMV launch,
+    chain mode runs every step in the persistent kernel with the per-step
+    handles; each step against the oracle on its actual input."""
+    M, T = 4, 4
+    lins = (synth.Linear("s0", 2048, 2048, 32, 64, 0), synth.Linear("s1", 2048, 2048, 32, 64, 1))
+    wl = synth.Workload("slt_decode", M=M, T=T, linears=lins, a_bits=8, outlier_frac=0.02,
+                        outlier_mult=20.0, x_dtype="bf16", description="SLT decode stack")
+    params = synth.module_params(wl)
+    shared = make_layer(params[1], 8)
+    own = [make_layer(q, 8) for q in _slt_params(params[0], T, 11)]
+    tl = [[own[t], shared] for t in range(T)]
+    handles = [[h[0] for h in row] for row in tl]
+    lq.lq_probe_enable(True)
+    try:
+        if mode == "open":
+            xs, flat = _stack_inputs(wl, M)
+            y = host(lq.lq_loop_stack_slt(act_tensor(flat, "bf16"), handles, lq.LQ_OPEN, M=M))
+        else:
+            x0 = synth.loop_input(wl, lins[0], 0)
+            y = host(lq.lq_loop_stack_slt(act_tensor(x0, "bf16"), handles, lq.LQ_CHAIN, M=M))
+        torch.cuda.synchronize()
+        probe = lq.lq_probe_read()
+    finally:
+        lq.lq_probe_enable(False)
+    if mode == "open":
+        assert probe["rotate_quantize"][1] == 1 and probe["gemv"][1] == 1, probe
+    else:
+        assert probe["chain_decode"][1] == 1 and probe["gemv"][1] == 0, probe
+    off = 0
+    xin, xdt = (None, "bf16") if mode == "open" else (x0, "bf16")
+    for t in range(T):
+        for l in range(2):
+            layer, ol = tl[t][l]
+            yg = y[off:off + M * 2048].reshape(M, 2048)
+            off += M * 2048
+            x = xs[t][l] if mode == "open" else xin
+            q8, _, sc = lq.lq_quantize_act(act_tensor(x, xdt), dev(ol.P1), dev(ol.P2),
+                                           float(ol.las[t]), 8)
+            torch.cuda.synchronize()
+            linear_parity(yg, x, ol, t, host(q8), host(sc), layer.w_flips)
+            if mode == "chain":
+                xin, xdt = yg, "f32"
+
+
 def test_loop_stack_slt_rejects_shape_mismatch():
     wl = synth.MLP
     params = synth.module_params(wl)
