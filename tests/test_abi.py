@@ -120,6 +120,17 @@ def test_loop_entry_points_reject_bad_arguments(L):
         lq.LQ_ERR_ARG
 
 
+def test_selftests_reject_bad_arguments(L):
+    """Both failure-path self-tests check their limit (and the grid wait its
+    scratch) before any launch."""
+    fake = 1 << 20
+    for bad in (0, -1, 10**8):
+        assert L.lq_selftest_bounded_wait(bad, None) == lq.LQ_ERR_ARG
+        assert L.lq_selftest_grid_wait(bad, fake, None) == lq.LQ_ERR_ARG
+    assert L.lq_selftest_grid_wait(1000, None, None) == lq.LQ_ERR_ARG
+    assert L.lq_selftest_grid_wait(1000, fake + 2, None) == lq.LQ_ERR_ARG  # misaligned
+
+
 def test_inverse_transpose_host_helper():
     rng = np.random.default_rng(0)
     for n in (1, 4, 16, 88):
