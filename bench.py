@@ -501,15 +501,25 @@ def e2e_measure(lq, ctx, wl, layers, x_dev, y_dev, ws, n_steps):
     while Mc > 16384 and Mc % 2 == 0:
         Mc //= 2
     n_chunks = M // Mc
-    # host input: the whole step, page-locked in place (exact size)
-    x_host = torch.empty(x_dev.numel(), dtype=x_dev.dtype)
+    # host input: the whole step, page-locked in place (exact size), unless the
+    # ranks of this node would pin more than about 60 % of the free host memory;
+    # then a two-chunk page-locked input ring whose chunks are sent again each
+    # time (the same bytes cross the bus per step; the outputs are not checked)
+    import psutil
+    local = int(os.environ.get("LOCAL_WORLD_SIZE", ctx.world))
+    nbytes = x_dev.numel() * x_el
+    pinned = nbytes + 2 * Mc * row_out * 4
+    in_ring = n_chunks > 2 and pinned * local > 0.6 * psutil.virtual_memory().available
+    x_host = torch.empty(2 * Mc * row_in if in_ring else x_dev.numel(), dtype=x_dev.dtype)
     cudart = torch.cuda.cudart()
-    nbytes = x_host.numel() * x_el
-    assert int(cudart.cudaHostRegister(x_host.data_ptr(), nbytes, 0)) == 0
+    assert int(cudart.cudaHostRegister(x_host.data_ptr(), x_host.numel() * x_el, 0)) == 0
     y_ring = torch.empty(2 * Mc * row_out, dtype=torch.float32)
     assert int(cudart.cudaHostRegister(y_ring.data_ptr(), y_ring.numel() * 4, 0)) == 0
     try:
-        x_host.copy_(x_dev)
+        if in_ring:
+            x_host.copy_(x_dev[:x_host.numel()])
+        else:
+            x_host.copy_(x_dev)
         slots = 1 if n_chunks == 1 else 2
         if n_chunks == 1:  # one chunk per step: separate device buffers, pipelined across steps
             xs = [x_dev, torch.empty_like(x_dev)]
@@ -536,6 +546,9 @@ def e2e_measure(lq, ctx, wl, layers, x_dev, y_dev, ws, n_steps):
             return out
 
         in_blocks = [blocks(c * Mc, Mc, row_in, Ks) for c in range(n_chunks)]
+        if in_ring:  # chunk c reads ring slot c % 2 (laid out as a chunk's blocks)
+            in_blocks = [[((c % 2) * Mc * row_in + coff, coff, ln) for _, coff, ln in blk]
+                         for c, blk in enumerate(in_blocks)]
         out_blocks = [blocks(0, Mc, row_out, Ns) for _ in range(1)][0]
 
         def run(n):
@@ -588,8 +601,10 @@ def e2e_measure(lq, ctx, wl, layers, x_dev, y_dev, ws, n_steps):
             "pipeline": f"{n_chunks} chunk(s) of {Mc} rows per step on two device buffer "
                         "sets; input copy of chunk i+1 and output copy of chunk i-1 overlap "
                         "chunk i's kernels",
-            "host_buffers": "whole-step input page-locked; outputs into a two-chunk "
-                            "page-locked host ring"}
+            "host_buffers": ("two-chunk page-locked input ring (host memory would not hold "
+                             "every rank's whole-step input)" if in_ring else
+                             "whole-step input page-locked") +
+                            "; outputs into a two-chunk page-locked host ring"}
 
 
 def measure_stack(lq, ctx, wl, n_steps, warmup, n_probe, peaks, want_clocks=False):
