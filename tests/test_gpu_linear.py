@@ -519,13 +519,19 @@ def test_loop_stack_chain_tiny():
                    what=f"chain t={t}")
 
 
-def _chain_decode_case(M, a_bits, x_dtype, T):
+def _chain_decode_case(M, a_bits, x_dtype, T, wide=False):
     """Three chained linears 2048 -> 1024 -> 3072 -> 2048 (factors 32x64,
-    32x32, 32x96), T loops with their own clips; returns the built layers,
-    the first input and the GPU outputs of the chain-mode stack with the probe
-    counts."""
-    lins = (synth.Linear("c0", 2048, 1024, 32, 64, 0), synth.Linear("c1", 1024, 3072, 32, 32, 1),
-            synth.Linear("c2", 3072, 2048, 32, 96, 2))
+    32x32, 32x96), or with `wide` 4096 -> 2048 -> 1024 -> 4096 (64x64, 32x64,
+    32x32), T loops with their own clips; returns the built layers, the first
+    input and the GPU outputs of the chain-mode stack with the probe counts."""
+    if wide:
+        lins = (synth.Linear("w0", 4096, 2048, 64, 64, 0),
+                synth.Linear("w1", 2048, 1024, 32, 64, 1),
+                synth.Linear("w2", 1024, 4096, 32, 32, 2))
+    else:
+        lins = (synth.Linear("c0", 2048, 1024, 32, 64, 0),
+                synth.Linear("c1", 1024, 3072, 32, 32, 1),
+                synth.Linear("c2", 3072, 2048, 32, 96, 2))
     wl = synth.Workload(f"chain_M{M}", M=M, T=T, linears=lins, a_bits=a_bits,
                         outlier_frac=0.02, outlier_mult=20.0, x_dtype=x_dtype,
                         description="chain-mode decode stack")
@@ -545,14 +551,18 @@ def _chain_decode_case(M, a_bits, x_dtype, T):
     return lins, params, built, x0, host(y), probe
 
 
-@pytest.mark.parametrize("M,a_bits,x_dtype,T", [(1, 8, "bf16", 4), (3, 4, "f32", 4),
-                                                (4, 8, "bf16", 4), (4, 4, "bf16", 43)])
-def test_loop_stack_chain_decode_persistent(M, a_bits, x_dtype, T):
+@pytest.mark.parametrize("M,a_bits,x_dtype,T,wide", [(1, 8, "bf16", 4, False),
+                                                     (3, 4, "f32", 4, False),
+                                                     (4, 8, "bf16", 4, False),
+                                                     (4, 4, "bf16", 43, False),
+                                                     (2, 8, "bf16", 4, True)])
+def test_loop_stack_chain_decode_persistent(M, a_bits, x_dtype, T, wide):
     """Decode-sized chain mode runs every step in the persistent kernel (one
-    launch per 128 steps, grid barriers between each step's quantize and GEMV):
-    each step's output against the oracle applied to the step's actual input
-    (the stack's input, then the previous step's float32 output)."""
-    lins, params, built, x0, y, probe = _chain_decode_case(M, a_bits, x_dtype, T)
+    launch per 128 steps; the quantize and the GEMV of a step handed over
+    through step counters): each step's output against the oracle applied to
+    the step's actual input (the stack's input, then the previous step's
+    float32 output).  Factor shapes 32x32 to 64x64 (K = 1024 to 4096)."""
+    lins, params, built, x0, y, probe = _chain_decode_case(M, a_bits, x_dtype, T, wide)
     L = len(lins)
     n_launch = -(-(T * L) // 128)
     assert probe["chain_decode"][1] == n_launch and probe["gemv"][1] == 0, probe
