@@ -311,25 +311,27 @@ def test_loop_stack_open_decode_branches(M, a_bits):
 @pytest.mark.parametrize("M,T,copies,a_bits,x_dtype", [
     (5, 4, 1, 8, "bf16"),    # loop batches of 3 and 1 (15 and 5 rows) in one launch
     (2, 4, 1, 4, "f32"),     # 8 rows: one token block
-    (16, 4, 9, 8, "bf16"),   # 108 units of one loop: two rounds of 54
+    (16, 4, 7, 8, "bf16"),   # 112 units of one loop: two rounds of 56
 ])
 def test_loop_stack_open_decode_grouped(M, T, copies, a_bits, x_dtype):
     """Decode-sized open mode with the stack's own workspace size: every
     (layer, loop batch) unit of a round in one quantize launch and one GEMV
     launch (two launches per round, counted by the probe), each unit with its
     own rows (ragged loop batches share a launch), layers of different widths
-    including a ragged N; every output of every loop against the oracle."""
+    (factors 16x32 to 64x88) including a ragged N; every output of every loop
+    against the oracle."""
     lins = (synth.Linear("g0", 512, 256, 16, 32, 0), synth.Linear("g1", 2048, 1000, 32, 64, 1),
-            synth.Linear("g2", 1024, 96, 32, 32, 2))
+            synth.Linear("g2", 1024, 96, 32, 32, 2), synth.Linear("g3", 5632, 200, 64, 88, 3))
+    nl = len(lins)
     wl = synth.Workload(f"decode_grouped_M{M}", M=M, T=T, linears=lins, a_bits=a_bits,
                         outlier_frac=0.02, outlier_mult=20.0, x_dtype=x_dtype,
                         description="grouped decode stack")
     params = synth.module_params(wl)
     built = [make_layer(mp, a_bits) for mp in params]
-    # the stack repeats the three linears `copies` times (same handles)
-    L = 3 * copies
-    layers = [built[l % 3][0] for l in range(L)]
-    xs = [[synth.loop_input(wl, lins[l % 3], t, rows=np.arange(M) + M * (l // 3))
+    # the stack repeats the four linears `copies` times (same handles)
+    L = nl * copies
+    layers = [built[l % nl][0] for l in range(L)]
+    xs = [[synth.loop_input(wl, lins[l % nl], t, rows=np.arange(M) + M * (l // nl))
            for l in range(L)] for t in range(T)]
     flat = np.concatenate([xs[t][l].ravel() for t in range(T) for l in range(L)])
     xd = act_tensor(flat, x_dtype)
@@ -349,15 +351,15 @@ def test_loop_stack_open_decode_grouped(M, T, copies, a_bits, x_dtype):
     off = 0
     for t in range(T):
         for l in range(L):
-            lin, mp = lins[l % 3], params[l % 3]
+            lin, mp = lins[l % nl], params[l % nl]
             n = M * lin.N
             yg = yh[off:off + n].reshape(M, lin.N)
             off += n
             q8, _, s = lq.lq_quantize_act(act_tensor(xs[t][l], x_dtype), dev(mp.P1),
                                           dev(mp.P2), float(mp.las[t]), a_bits)
             torch.cuda.synchronize()
-            linear_parity(yg, xs[t][l], built[l % 3][1], t, host(q8), host(s),
-                          built[l % 3][0].w_flips)
+            linear_parity(yg, xs[t][l], built[l % nl][1], t, host(q8), host(s),
+                          built[l % nl][0].w_flips)
 
 
 def test_loop_stack_open_more_than_eight_loops():
