@@ -1039,15 +1039,17 @@ __global__ void __launch_bounds__(kThreads) k_rotate_quant_small(
 //  1. every block starts copying its slice of the step's weights (rows
 //     [n0, n1) of N: packed codes and steps, both contiguous in memory) into
 //     shared memory with cp.async, not waited for yet;
-//  2. blocks 0 .. M * b/32 - 1 stage their factors, wait until every block
-//     has written the previous step's output (a counter of blocks), then
-//     rotate and quantize one (row, 32-column slice) of the step's input each
-//     (the few-row block above), write the activation codes (kOpGemvAct
-//     layout), steps and group sums, and count themselves done;
+//  2. blocks 0 .. M * b/32 - 1 widen their factors (copied raw during the
+//     previous step) into float64 operands, wait until every block has
+//     written the previous step's output (a counter of blocks), then rotate
+//     and quantize one (row, 32-column slice) of the step's input each (the
+//     few-row block above), write the activation codes (kOpGemvAct layout),
+//     steps and group sums, count themselves done, and start copying the
+//     next step's factors;
 //  3. every block waits for the step's quantize blocks (a second counter),
 //     copies the activation into shared memory, waits for its weight rows
-//     and forms y[m][n] for them: warp per weight row, lane per group, dp4a
-//     on the offset-binary nibbles minus 8 * sum q_a, the fold with both
+//     and forms y[m][n] for them: two weight rows per warp, lane per group,
+//     dp4a on the offset-binary nibbles minus 8 * sum q_a, the fold with both
 //     steps in float32, a butterfly sum over the lanes per token (the same
 //     arithmetic, in the same order, as the dp4a GEMV kernel), and counts
 //     itself done.
